@@ -1,0 +1,485 @@
+"""Pins for the fp64 CPU oracle: each test checks the oracle against something
+other than itself -- a closed form, a property the pages state, a brute force
+on tiny inputs, or an independent implementation of a published definition.
+
+Sources: "Speculative Speculative Decoding" (gist.science, Chinese and Dutch
+editions), technical summary sections 2 and 3; Salmon et al., "Parallel Random
+Numbers: As Easy as 1, 2, 3" (SC'11) for Philox.
+"""
+import itertools
+
+import numpy as np
+import pytest
+
+import oracle
+from speculative_decoding_verify_ssd_b200 import synth
+
+GRID = 1 << 24  # uniforms are m * 2^-24, m in [0, 2^24)
+
+
+def softmax64(l, T):
+    x = np.asarray(l, dtype=np.float64) / T
+    e = np.exp(x - x.max())
+    return e / e.sum()
+
+
+def grid_u(m):
+    return (np.asarray(m, dtype=np.float64) / GRID).astype(np.float32)
+
+
+def grid_bisect(pred, n):
+    """Smallest m in [0, GRID] with pred(m) False, for n monotone predicates
+    (True below the breakpoint).  pred takes an int64 array of length n."""
+    lo = np.zeros(n, dtype=np.int64)        # pred(lo) assumed True (or lo == breakpoint)
+    hi = np.full(n, GRID, dtype=np.int64)   # GRID stands for "never False"
+    first = pred(lo)
+    lo_done = ~first                        # already False at m = 0
+    while np.any((hi - lo > 1) & ~lo_done):
+        mid = (lo + hi) // 2
+        ok = pred(mid)
+        lo = np.where(ok & ~lo_done, mid, lo)
+        hi = np.where(~ok & ~lo_done, mid, hi)
+    return np.where(lo_done, 0, hi)
+
+
+def tile_rows(x, n):
+    return np.ascontiguousarray(np.broadcast_to(x, (n,) + x.shape))
+
+
+class Case:
+    """One fixed row of small logits, replicated over a batch of probes."""
+
+    def __init__(self, lp, lq, T, F, C, budget):
+        self.lp, self.lq, self.T, self.F, self.C, self.budget = lp, lq, T, F, C, budget
+        self.K = lq.shape[0]
+        self.V = lq.shape[1]
+
+    def verify(self, D, U, **kw):
+        n = D.shape[0]
+        F = None if self.F is None else tile_rows(self.F, n)
+        return oracle.verify(tile_rows(self.lp, n), tile_rows(self.lq, n), D, U, self.T, F=F,
+                             C_coef=self.C, budget=self.budget, n_threads=1, **kw)
+
+    def sample(self, Ud):
+        n = Ud.shape[0]
+        return oracle.reweight(tile_rows(self.lq, n), self.T, tile_rows(self.F, n), self.C,
+                               self.budget, u_draft=Ud, n_threads=1)["tokens"]
+
+    def draft_dist(self):
+        """q'_j measured from the oracle's own draft sampler (inverse CDF)."""
+        K, V = self.K, self.V
+        jj, vv = np.meshgrid(np.arange(K), np.arange(V - 1), indexing="ij")
+        jj, vv = jj.ravel(), vv.ravel()
+
+        def pred(m):
+            Ud = np.zeros((m.size, K), np.float32)
+            Ud[np.arange(m.size), jj] = grid_u(m)
+            tok = self.sample(Ud)
+            return tok[np.arange(m.size), jj] <= vv
+
+        beta = grid_bisect(pred, jj.size).reshape(K, V - 1)
+        edges = np.concatenate([np.zeros((K, 1), np.int64), beta, np.full((K, 1), GRID)], axis=1)
+        return np.diff(edges, axis=1) / GRID
+
+    def accept_grid(self):
+        """A_j(v): fraction of the uniform grid on which token v is accepted at j."""
+        K, V = self.K, self.V
+        jj, vv = np.meshgrid(np.arange(K), np.arange(V), indexing="ij")
+        jj, vv = jj.ravel(), vv.ravel()
+
+        def pred(m):
+            D = np.zeros((m.size, K), np.int32)
+            D[np.arange(m.size), jj] = vv
+            U = np.zeros((m.size, K + 1), np.float32)
+            U[np.arange(m.size), jj] = grid_u(m)
+            out = self.verify(D, U)
+            return out["n_accepted"] > jj
+
+        return (grid_bisect(pred, jj.size) / GRID).reshape(K, V)
+
+    def bonus_dist(self, k, d_reject):
+        """Distribution of the bonus token when k* = k (k < K: rejection at k
+        with draft token d_reject; k = K: full acceptance)."""
+        K, V = self.K, self.V
+        vv = np.arange(V - 1)
+
+        def pred(m):
+            D = np.zeros((m.size, K), np.int32)
+            U = np.zeros((m.size, K + 1), np.float32)
+            if k < K:
+                D[:, k] = d_reject
+                U[:, k] = np.float32((GRID - 1) / GRID)
+            U[:, K] = grid_u(m)
+            out = self.verify(D, U)
+            assert np.all(out["n_accepted"] == k)
+            return out["bonus"] <= vv
+
+        beta = grid_bisect(pred, V - 1)
+        edges = np.concatenate([[0], beta, [GRID]])
+        return np.diff(edges) / GRID
+
+
+def make_case(K, V, T, C, seed, budget=6, alpha=0.6, draft_scale=1.0):
+    rng = np.random.default_rng(seed)
+    lp = rng.normal(0.0, 1.5, (K + 1, V)).astype(np.float32)
+    lq = (lp[:K] + rng.normal(0.0, draft_scale, (K, V))).astype(np.float32)
+    F = oracle.fanout_plan(alpha, K, budget)
+    return Case(lp, lq, T, F, C, budget)
+
+
+# ---------------------------------------------------------------------------
+# Losslessness: the whole draft-sample + verify step reproduces p exactly.
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("K", [2, 3])
+@pytest.mark.parametrize("C", [1.0, 0.5, 0.2])
+@pytest.mark.parametrize("T", [1.0, 0.7])
+def test_lossless_by_enumeration(K, C, T):
+    """[ZH] section 2 / [NL] section 2: the method is lossless.  With d_j drawn
+    by the oracle's Saguaro sampler and every uniform on the 2^-24 grid
+    enumerated interval by interval, the token emitted at each position j,
+    given that position j is reached, is distributed exactly as p_j."""
+    case = make_case(K, 8, T, C, seed=10 * K + int(C * 10))
+    qp = case.draft_dist()
+    A = case.accept_grid()
+    for j in range(K + 1):
+        p = softmax64(case.lp[j], T)
+        if j < K:
+            rej_tok = int(np.argmin(A[j]))
+            g = case.bonus_dist(j, rej_tok) if A[j, rej_tok] < 1.0 else np.zeros(case.V)
+            emitted = qp[j] * A[j] + np.sum(qp[j] * (1.0 - A[j])) * g
+        else:
+            emitted = case.bonus_dist(K, None)
+        np.testing.assert_allclose(emitted, p, atol=2e-6, rtol=0)
+        assert abs(emitted.sum() - 1.0) < 2e-6
+
+
+def test_lossless_detects_plain_q_in_accept_test():
+    """The enumeration is sensitive: drafting from q' but scoring against q
+    (a plausible slip) breaks losslessness for C < 1, so the check above would
+    catch it.  Here the mistake is planted in the test's own composition."""
+    case = make_case(2, 8, 1.0, 0.3, seed=7)
+    qp = case.draft_dist()
+    q = softmax64(case.lq[0], 1.0)
+    p = softmax64(case.lp[0], 1.0)
+    a_wrong = np.minimum(1.0, p / q)
+    r = np.maximum(0.0, p - q)
+    emitted = qp[0] * a_wrong + np.sum(qp[0] * (1 - a_wrong)) * r / r.sum()
+    assert np.max(np.abs(emitted - p)) > 1e-3
+
+
+# ---------------------------------------------------------------------------
+# Saguaro sampling: the structure the pages describe, measured from the sampler.
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("C", [1.0, 0.6, 0.25])
+def test_saguaro_downweights_topF_by_C(C):
+    """[ZH] section 2 challenge 2 / [NL] section 3B: the draft's top-F tokens
+    are down-weighted by C and the distribution renormalised.  Measured q'
+    must equal q scaled by C/Z on the top-F set and by 1/Z elsewhere, with S
+    the top-F of the raw logits (brute-force sort)."""
+    K, V = 2, 12
+    case = make_case(K, V, 0.8, C, seed=3, budget=7, alpha=0.5)
+    qp = case.draft_dist()
+    for j in range(K):
+        q = softmax64(case.lq[j], 0.8)
+        S = sorted(range(V), key=lambda v: (-float(case.lq[j, v]), v))[: case.F[j]]
+        w = np.ones(V)
+        w[S] = C
+        expect = w * q / np.sum(w * q)
+        np.testing.assert_allclose(qp[j], expect, atol=2e-6, rtol=0)
+
+
+def test_saguaro_C1_is_identity_and_outputs_match_unweighted():
+    case = make_case(3, 16, 1.0, 1.0, seed=5, budget=9)
+    rng = np.random.default_rng(1)
+    n = 64
+    D = rng.integers(0, 16, (n, 3)).astype(np.int32)
+    U = synth.uniforms(11, n, 4, 0)
+    with_plan = case.verify(D, U)
+    plain = Case(case.lp, case.lq, 1.0, None, 1.0, 0).verify(D, U)
+    assert np.all(with_plan["Z"] == 1.0)
+    for key in ("n_accepted", "bonus", "out_tokens"):
+        np.testing.assert_array_equal(with_plan[key], plain[key])
+    np.testing.assert_array_equal(with_plan["accept_prob"], plain["accept_prob"])
+
+
+def test_saguaro_raises_bonus_mass_on_cached_set():
+    """[ZH] section 2 challenge 2: lowering C moves residual mass onto the
+    cached top-F tokens, so the bonus lands in S more often (at rejection)."""
+    K, V = 2, 10
+    masses = []
+    for C in (1.0, 0.7, 0.4, 0.1):
+        case = make_case(K, V, 1.0, C, seed=21, budget=6, alpha=0.5)
+        A = case.accept_grid()
+        tok = int(np.argmin(A[0]))
+        g = case.bonus_dist(0, tok)
+        S = sorted(range(V), key=lambda v: (-float(case.lq[0, v]), v))[: case.F[0]]
+        masses.append(g[S].sum())
+    assert all(masses[i] <= masses[i + 1] + 1e-7 for i in range(len(masses) - 1)), masses
+    assert masses[-1] > masses[0] + 0.05
+
+
+# ---------------------------------------------------------------------------
+# Identities.
+# ---------------------------------------------------------------------------
+def test_q_equals_p_accepts_everything():
+    rng = np.random.default_rng(2)
+    K, V, n = 4, 50, 200
+    lp = rng.normal(0, 2, (K + 1, V)).astype(np.float32)
+    case = Case(lp, lp[:K].copy(), 1.0, oracle.fanout_plan(0.7, K, 10), 1.0, 10)
+    D = rng.integers(0, V, (n, K)).astype(np.int32)
+    U = synth.uniforms(3, n, K + 1, 0)
+    out = case.verify(D, U)
+    assert np.all(out["n_accepted"] == K)
+    assert np.all(out["accept_prob"] == 1.0)
+
+
+def test_residual_mass_identity():
+    """R = sum max(0, p - q') = 1 - sum min(p, q'), with q' measured from the
+    sampler and p from the definition."""
+    case = make_case(2, 8, 1.0, 0.4, seed=9)
+    qp = case.draft_dist()
+    A = case.accept_grid()
+    tok = int(np.argmin(A[1]))
+    D = np.zeros((1, 2), np.int32)
+    D[0, 1] = tok
+    U = np.zeros((1, 3), np.float32)
+    U[0, 1] = np.float32((GRID - 1) / GRID)
+    out = case.verify(D, U)
+    assert out["n_accepted"][0] == 1
+    p = softmax64(case.lp[1], 1.0)
+    assert abs(out["residual_mass"][0] - (1.0 - np.minimum(p, qp[1]).sum())) < 2e-6
+
+
+def test_accept_prob_matches_grid_and_ratio_bound():
+    case = make_case(3, 8, 1.0, 0.5, seed=4)
+    A = case.accept_grid()
+    n = 8
+    D = np.tile(np.arange(8, dtype=np.int32)[:, None], (1, 3))
+    out = case.verify(D, np.zeros((n, 4), np.float32))
+    a = out["accept_prob"]  # [8 tokens, 3 positions]
+    np.testing.assert_allclose(a.T, A, atol=1.0 / GRID + 1e-12)
+    assert np.all((a >= 0) & (a <= 1))
+
+
+# ---------------------------------------------------------------------------
+# Temperature 0: textbook greedy verification.
+# ---------------------------------------------------------------------------
+def test_greedy_is_textbook():
+    rng = np.random.default_rng(8)
+    K, V, n = 5, 40, 300
+    lp = np.round(rng.normal(0, 1, (n, K + 1, V)) * 4) / 4  # ties on purpose
+    lp = lp.astype(np.float32)
+    lq = (lp[:, :K] + rng.normal(0, 0.5, (n, K, V))).astype(np.float32)
+    am = np.argmax(lp, axis=2)  # numpy: first index of the maximum
+    D = np.where(rng.random((n, K)) < 0.8, am[:, :K], rng.integers(0, V, (n, K))).astype(np.int32)
+    U = synth.uniforms(5, n, K + 1, 0)
+    F = np.tile(oracle.fanout_plan(0.7, K, 12), (n, 1))
+    out = oracle.verify(lp, lq, D, U, 0.0, F=F, C_coef=0.5, budget=12, n_threads=2)
+    for b in range(n):
+        mism = [j for j in range(K) if D[b, j] != am[b, j]]
+        k = mism[0] if mism else K
+        assert out["n_accepted"][b] == k
+        assert out["bonus"][b] == am[b, k]
+        assert list(out["out_tokens"][b]) == list(D[b, :k]) + [am[b, k]] + [-1] * (K - k)
+        assert np.all(out["Z"][b] == 1.0)
+
+
+# ---------------------------------------------------------------------------
+# Top-F and the cache.
+# ---------------------------------------------------------------------------
+def brute_topf(x, F):
+    return [v for v in sorted(range(len(x)), key=lambda v: (-float(x[v]), v))][:F]
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_topf_matches_brute_force_with_ties(seed):
+    rng = np.random.default_rng(seed)
+    V = int(rng.integers(1, 300))
+    x = synth.bf16_bits_to_f32(synth.f32_to_bf16_bits(np.round(rng.normal(0, 1, V) * 3) / 3))
+    x = x.astype(np.float64)
+    x[rng.random(V) < 0.1] = -np.inf
+    z = rng.random(V) < 0.1
+    x[z] = np.where(rng.random(z.sum()) < 0.5, -0.0, 0.0)
+    for F in sorted({0, 1, min(5, V), V // 2, V}):
+        assert list(oracle.topf(x, F)) == brute_topf(x, F)
+
+
+def test_cache_segments_are_topf_sets():
+    rng = np.random.default_rng(12)
+    B, K, V, budget = 6, 3, 64, 11
+    lp = rng.normal(0, 1, (B, K + 1, V)).astype(np.float32)
+    lq = (lp[:, :K] + rng.normal(0, 0.7, (B, K, V))).astype(np.float32)
+    ln = rng.normal(0, 1, (B, V)).astype(np.float32)
+    F = np.stack([oracle.fanout_plan(a, K, budget) for a in (0.2, 0.5, 0.9, 0.6, 0.7, 0.99)])
+    D = rng.integers(0, V, (B, K)).astype(np.int32)
+    U = synth.uniforms(1, B, K + 1, 0)
+    for nxt in (None, ln):
+        out = oracle.verify(lp, lq, D, U, 1.0, F=F, C_coef=0.5, budget=budget, draft_next=nxt)
+        for b in range(B):
+            off = out["offsets"][b]
+            assert list(off) == [0] + list(np.cumsum(F[b]))
+            for k in range(K + 1):
+                src = lq[b, k] if k < K else (ln[b] if nxt is not None else lp[b, K])
+                seg = out["cache_tokens"][b, off[k]:off[k + 1]]
+                assert list(seg) == brute_topf(src, F[b, k])
+            k = out["n_accepted"][b]
+            seg = list(out["cache_tokens"][b, off[k]:off[k + 1]])
+            bon = out["bonus"][b]
+            assert out["hit"][b] == (bon in seg)
+            assert out["slot"][b] == (off[k] + seg.index(bon) if bon in seg else -1)
+
+
+def test_lookup_brute_force():
+    rng = np.random.default_rng(13)
+    B, K, budget, V = 50, 4, 20, 1000
+    offsets = np.zeros((B, K + 2), np.int32)
+    tokens = np.zeros((B, budget), np.int32)
+    for b in range(B):
+        cuts = np.sort(rng.integers(0, budget + 1, K))
+        offsets[b] = np.concatenate([[0], cuts, [budget]])
+        tokens[b] = rng.choice(V, budget, replace=False)
+    k = rng.integers(0, K + 1, B).astype(np.int32)
+    bonus = np.where(rng.random(B) < 0.5, tokens[np.arange(B), rng.integers(0, budget, B)],
+                     rng.integers(0, V, B)).astype(np.int32)
+    payload = rng.integers(0, V, (B, budget, K)).astype(np.int32)
+    out = oracle.cache_lookup(offsets, tokens, k, bonus, V, payload=payload, fallback_seed=77)
+    for b in range(B):
+        seg = list(tokens[b, offsets[b, k[b]]:offsets[b, k[b] + 1]])
+        if bonus[b] in seg:
+            s = offsets[b, k[b]] + seg.index(bonus[b])
+            assert out["hit"][b] == 1 and out["slot"][b] == s
+            assert list(out["next_tokens"][b]) == list(payload[b, s])
+        else:
+            assert out["hit"][b] == 0 and out["slot"][b] == -1
+            words = synth.philox4x32_10(np.array([[b, i, 2, 0] for i in range(K)], np.uint32),
+                                        synth.seed_key(77))[:, 0]
+            expect = (words.astype(np.uint64) * np.uint64(V)) >> np.uint64(32)
+            assert list(out["next_tokens"][b]) == list(expect.astype(np.int32))
+
+
+# ---------------------------------------------------------------------------
+# Fan-out plan.
+# ---------------------------------------------------------------------------
+def test_fanout_worked_examples():
+    """Hand-derived from the geometric reading (not printed on the pages):
+    alpha = 0.7 quotas rounded by largest remainder."""
+    assert list(oracle.fanout_plan(0.7, 6, 64)) == [19, 13, 9, 7, 5, 3, 8]
+    assert list(oracle.fanout_plan(0.7, 4, 8)) == [2, 2, 1, 1, 2]
+    assert list(oracle.fanout_plan(0.7, 8, 128)) == [38, 27, 19, 13, 9, 7, 5, 3, 7]
+
+
+def test_fanout_extremes_and_uniform():
+    assert list(oracle.fanout_plan(0.0, 5, 30)) == [30, 0, 0, 0, 0, 0]
+    assert list(oracle.fanout_plan(1.0, 5, 30)) == [0, 0, 0, 0, 0, 30]
+    assert list(oracle.fanout_plan(0.3, 6, 64, mode=1)) == [10, 9, 9, 9, 9, 9, 9]
+    assert list(oracle.fanout_plan(0.3, 3, 0)) == [0, 0, 0, 0]
+
+
+def quotas(alpha, K, budget):
+    P = [alpha ** k * (1 - alpha) for k in range(K)] + [alpha ** K]
+    return [budget * p for p in P]
+
+
+def test_fanout_sum_rank_and_quota_bounds():
+    rng = np.random.default_rng(0)
+    for _ in range(400):
+        K = int(rng.integers(1, 12))
+        budget = int(rng.integers(0, 300))
+        alpha = float(np.float32(rng.random()))
+        F = oracle.fanout_plan(alpha, K, budget)
+        Q = quotas(alpha, K, budget)
+        assert F.sum() == budget and np.all(F >= 0)
+        for a, b in itertools.combinations(range(K + 1), 2):
+            if Q[a] > Q[b] + 1e-9:
+                assert F[a] >= F[b]
+        assert all(abs(F[k] - Q[k]) < 1.0 + 1e-9 for k in range(K + 1))
+        if 0 < alpha < 1:   # geometric: successive quota ratio alpha for k+1 < K
+            for k in range(K - 1):
+                assert abs(Q[k + 1] / Q[k] - alpha) < 1e-12 if Q[k] > 0 else True
+
+
+def test_fanout_largest_remainder_is_optimal_apportionment():
+    """Brute force: among all integer splits of the budget, the plan minimises
+    the total absolute deviation from the quotas."""
+    for alpha in (0.15, 0.5, 0.73, 0.9):
+        for K in (1, 2, 3):
+            for budget in range(0, 11):
+                Q = np.array(quotas(alpha, K, budget))
+                F = oracle.fanout_plan(alpha, K, budget)
+                best = min(np.abs(np.array(c) - Q).sum()
+                           for c in itertools.product(range(budget + 1), repeat=K + 1)
+                           if sum(c) == budget)
+                assert np.abs(F - Q).sum() <= best + 1e-9
+
+
+# ---------------------------------------------------------------------------
+# Philox4x32-10 and the uniform / fallback encodings.
+# ---------------------------------------------------------------------------
+def test_philox_two_implementations_agree():
+    rng = np.random.default_rng(0)
+    ctr = rng.integers(0, 2 ** 32, (20000, 4), dtype=np.uint64).astype(np.uint32)
+    key = rng.integers(0, 2 ** 32, (20000, 2), dtype=np.uint64).astype(np.uint32)
+    np.testing.assert_array_equal(oracle.philox4x32_10(ctr, key), synth.philox4x32_10(ctr, key))
+
+
+def test_philox_statistics():
+    n = 1 << 18
+    ctr = np.stack([np.arange(n), np.zeros(n), np.zeros(n), np.zeros(n)], axis=1).astype(np.uint32)
+    out = oracle.philox4x32_10(ctr, np.array([123, 456], np.uint32))
+    assert len(np.unique(out[:, 0])) > n - 20        # a bijection of the counter
+    for w in range(4):
+        counts = np.bincount(out[:, w] >> 24, minlength=256)
+        chi2 = ((counts - n / 256) ** 2 / (n / 256)).sum()
+        assert chi2 < 400                             # 255 dof; p ~ 1e-8 tail
+    bits = np.unpackbits(out.view(np.uint8)).reshape(n, 128).mean(axis=0)
+    assert np.all(np.abs(bits - 0.5) < 0.01)
+
+
+def test_uniform_encoding_and_range():
+    u = synth.uniforms(5, 100, 7, 0)
+    assert u.dtype == np.float32 and np.all(u >= 0) and np.all(u < 1)
+    assert np.all(u * GRID == np.floor(u * GRID))
+    ctr = np.array([[3, 4, 0, 0]], np.uint32)
+    x = oracle.philox4x32_10(ctr, synth.seed_key(5))[0, 0]
+    assert u[3, 4] == np.float32((x >> 8) / GRID)
+
+
+# ---------------------------------------------------------------------------
+# Invalid inputs and the diagnostic hit probability.
+# ---------------------------------------------------------------------------
+def test_invalid_rows_are_flagged():
+    rng = np.random.default_rng(3)
+    B, K, V, budget = 5, 2, 32, 6
+    lp = rng.normal(0, 1, (B, K + 1, V)).astype(np.float32)
+    lq = rng.normal(0, 1, (B, K, V)).astype(np.float32)
+    D = rng.integers(0, V, (B, K)).astype(np.int32)
+    U = synth.uniforms(1, B, K + 1, 0)
+    F = np.tile(oracle.fanout_plan(0.5, K, budget), (B, 1))
+    lp[0, 1, 3] = np.nan
+    lq[1, 0, :] = -np.inf
+    D[2, 1] = V
+    U[3, 2] = 1.0
+    F[4, 0] += 1
+    out = oracle.verify(lp, lq, D, U, 1.0, F=F, C_coef=0.5, budget=budget, fallback_seed=9)
+    assert list(out["status"] & oracle.ROW_INVALID) == [oracle.ROW_NONFINITE, oracle.ROW_NONFINITE,
+                                                         oracle.ROW_BAD_TOKEN, oracle.ROW_BAD_UNIFORM,
+                                                         oracle.ROW_BAD_PLAN]
+    assert np.all(out["n_accepted"] == -1) and np.all(out["bonus"] == -1)
+    assert np.all(out["out_tokens"] == -1) and np.all(np.isnan(out["accept_prob"]))
+    assert np.all(out["hit"] == 0) and np.all(out["slot"] == -1)
+    assert np.all(out["cache_tokens"] == -1)
+
+
+def test_expected_hit_probability_matches_frequency():
+    rng = np.random.default_rng(17)
+    K, V, n, budget = 3, 24, 40000, 9
+    lp = rng.normal(0, 1.2, (K + 1, V)).astype(np.float32)
+    lq = (lp[:K] + rng.normal(0, 0.8, (K, V))).astype(np.float32)
+    case = Case(lp, lq, 1.0, oracle.fanout_plan(0.6, K, budget), 0.4, budget)
+    D = np.tile(np.array([[3, 7, 11]], np.int32), (n, 1))
+    U = synth.uniforms(23, n, K + 1, 0)
+    out = case.verify(D, U, want_phit=True)
+    ph = out["p_hit"][0]
+    assert np.allclose(out["p_hit"], ph)
+    freq = out["hit"].mean()
+    assert abs(freq - ph) < 4.5 * np.sqrt(ph * (1 - ph) / n) + 1e-9
