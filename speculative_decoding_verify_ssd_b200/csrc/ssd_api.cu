@@ -1,0 +1,396 @@
+// ssd_api.cu -- host side of libssd: argument checks, launch planning and the
+// extern "C" entry points declared in include/ssd.h, plus the three small
+// kernels (fan-out plan, cache build, cache lookup).
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+
+#include <map>
+#include <mutex>
+#include <tuple>
+
+#include "../../include/ssd.h"
+#include "ssd_device.cuh"
+#include "ssd_unit_kernel.cuh"
+
+namespace ssd {
+
+// ---------------------------------------------------------------------------
+// Fan-out plan ([ZH] section 2 challenge 1; [NL] section 3A).  fp64, every
+// product and difference rounded on its own (no fused multiply-add).
+// ---------------------------------------------------------------------------
+__global__ void fanout_kernel(const float* __restrict__ alpha, int B, int K, int budget, int mode,
+                              int32_t* __restrict__ F) {
+  const int b = blockIdx.x * blockDim.x + threadIdx.x;
+  if (b >= B) return;
+  fanout_row(mode == SSD_FANOUT_UNIFORM ? 0.f : alpha[b], K, budget, mode,
+             F + static_cast<long long>(b) * (K + 1));
+}
+
+// ---------------------------------------------------------------------------
+// Cache build: offsets = prefix sums of F; tokens copied per segment.
+// ---------------------------------------------------------------------------
+__global__ void cache_build_kernel(const int32_t* __restrict__ F, const int32_t* __restrict__ topf,
+                                   const int32_t* __restrict__ guess_K, int K, int budget,
+                                   int32_t* __restrict__ offsets, int32_t* __restrict__ tokens) {
+  __shared__ int32_t off[SSD_MAX_K + 2];
+  __shared__ int32_t bad;
+  const int b = blockIdx.x;
+  const int32_t* Fr = F + static_cast<long long>(b) * (K + 1);
+  if (threadIdx.x == 0) {
+    long long sum = 0;
+    int pb = 0;
+    for (int k = 0; k <= K; ++k) {
+      if (Fr[k] < 0) pb = 1;
+      sum += Fr[k];
+    }
+    if (sum != budget) pb = 1;
+    bad = pb;
+    off[0] = 0;
+    for (int k = 0; k <= K; ++k) off[k + 1] = off[k] + (pb ? 0 : Fr[k]);
+    for (int k = 0; k <= K + 1; ++k) offsets[static_cast<long long>(b) * (K + 2) + k] = off[k];
+  }
+  __syncthreads();
+  for (int s = threadIdx.x; s < budget; s += blockDim.x) {
+    int32_t t = -1;
+    if (!bad) {
+      if (guess_K && s >= off[K])
+        t = guess_K[static_cast<long long>(b) * budget + (s - off[K])];
+      else
+        t = topf[static_cast<long long>(b) * budget + s];
+    }
+    tokens[static_cast<long long>(b) * budget + s] = t;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Cache lookup ([ZH] section 2 basic flow step 4, challenge 3; [NL] 3C).
+// ---------------------------------------------------------------------------
+__global__ void cache_lookup_kernel(const int32_t* __restrict__ offsets, const int32_t* __restrict__ tokens,
+                                    int B, int K, int budget, const int32_t* __restrict__ k,
+                                    const int32_t* __restrict__ bonus, const int32_t* __restrict__ payload,
+                                    unsigned long long seed, int V, uint8_t* __restrict__ hit,
+                                    int32_t* __restrict__ slot, int32_t* __restrict__ next_tokens) {
+  const int b = blockIdx.x * blockDim.x + threadIdx.x;
+  if (b >= B) return;
+  const int kk = k[b];
+  const int32_t bon = bonus[b];
+  int sl = -1;
+  if (kk >= 0 && kk <= K) {
+    const int32_t* o = offsets + static_cast<long long>(b) * (K + 2);
+    const int lo = max(o[kk], 0), hi = min(o[kk + 1], budget);
+    for (int s = lo; s < hi; ++s)
+      if (tokens[static_cast<long long>(b) * budget + s] == bon) {
+        sl = s;
+        break;
+      }
+  }
+  hit[b] = sl >= 0 ? 1 : 0;
+  slot[b] = sl;
+  for (int i = 0; i < K; ++i) {
+    int32_t t;
+    if (sl >= 0)
+      t = payload ? payload[(static_cast<long long>(b) * budget + sl) * K + i] : -1;
+    else
+      t = fallback_token(seed, b, i, V);
+    next_tokens[static_cast<long long>(b) * K + i] = t;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Launch planning.
+// ---------------------------------------------------------------------------
+#ifndef SSD_CTA_BYTES
+#define SSD_CTA_BYTES 65536   // logits streamed per CTA per unit (all rows of the unit)
+#endif
+constexpr long long kCtaBytes = SSD_CTA_BYTES;
+constexpr int kMinChunk = 1024;  // do not split a row finer than this
+
+struct Plan {
+  int n_cta, chunk;
+  size_t smem;  // bulk-copy ring (aligned rows only)
+};
+
+static int sm_count() {
+  int dev = 0, n = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n > 0 ? n : 148;
+}
+
+// Cluster size and slice length for one unit of `rows` logit rows of length V.
+static ssd_status make_plan(int V, int rows, int esize, long long units, Plan* p) {
+  const int VE = 16 / esize;
+  const long long max_chunk = static_cast<long long>(kMaxChunks) * kChunkVecs * VE;
+  long long n_cta = (static_cast<long long>(rows) * V * esize + kCtaBytes - 1) / kCtaBytes;
+  // Enough CTAs to fill the machine, if the rows are long enough.
+  const long long want = (static_cast<long long>(kMinBlocks) * sm_count() + units - 1) / (units > 0 ? units : 1);
+  const long long by_len = (V + kMinChunk - 1) / kMinChunk;
+  long long extra = want < by_len ? want : by_len;
+  if (extra > 8) extra = 8;
+  if (n_cta < extra) n_cta = extra;
+  if (n_cta < 1) n_cta = 1;
+  long long chunk = (V + n_cta - 1) / n_cta;
+  chunk = (chunk + VE - 1) / VE * VE;
+  if (chunk > max_chunk) {
+    n_cta = (V + max_chunk - 1) / max_chunk;
+    chunk = (V + n_cta - 1) / n_cta;
+    chunk = (chunk + VE - 1) / VE * VE;
+  }
+  n_cta = (V + chunk - 1) / chunk;
+  if (n_cta > kMaxCluster) return SSD_ERR_UNSUPPORTED;
+  p->n_cta = static_cast<int>(n_cta);
+  p->chunk = static_cast<int>(chunk);
+  p->smem = static_cast<size_t>(kStages) * (rows > 1 ? 2 : 1) * kChunkVecs * 16;
+  return SSD_OK;
+}
+
+static std::mutex g_attr_mu;
+static std::map<std::tuple<const void*, int>, int> g_attr_done;
+
+static cudaError_t prepare_kernel(const void* fn, size_t smem) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lock(g_attr_mu);
+  auto key = std::make_tuple(fn, dev);
+  auto it = g_attr_done.find(key);
+  if (it != g_attr_done.end() && it->second >= static_cast<int>(smem)) return cudaSuccess;
+  // clusters of up to 16 CTAs; the bulk-copy ring in dynamic shared memory
+  e = cudaFuncSetAttribute(fn, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  g_attr_done[key] = static_cast<int>(smem);
+  return cudaSuccess;
+}
+
+struct WsLayout {
+  size_t units, counters, first_rej, error, total;
+};
+
+static WsLayout ws_layout(int B, int K) {
+  WsLayout w;
+  const size_t nb = static_cast<size_t>(B > 0 ? B : 0);
+  w.units = 0;
+  w.counters = w.units + nb * static_cast<size_t>(K + 1) * sizeof(UnitRes);
+  w.first_rej = w.counters + nb * sizeof(int32_t);
+  w.error = w.first_rej + nb * sizeof(int32_t);
+  w.total = (w.error + sizeof(int32_t) + 255) / 256 * 256;
+  return w;
+}
+
+static void bind_workspace(UnitArgs& a, void* ws, int B, int K) {
+  const WsLayout w = ws_layout(B, K);
+  char* base = static_cast<char*>(ws);
+  a.units = reinterpret_cast<UnitRes*>(base + w.units);
+  a.counters = reinterpret_cast<int32_t*>(base + w.counters);
+  a.first_rej = reinterpret_cast<int32_t*>(base + w.first_rej);
+  a.error = reinterpret_cast<int32_t*>(base + w.error);
+}
+
+template <typename TIn, bool kAligned, bool kGreedy>
+static ssd_status launch_units_t(const UnitArgs& a, const Plan& plan, long long units, cudaStream_t stream) {
+  const void* fn = reinterpret_cast<const void*>(&ssd_unit_kernel<TIn, kAligned, kGreedy>);
+  const size_t smem = kAligned ? plan.smem : 0;
+  if (prepare_kernel(fn, smem) != cudaSuccess) return SSD_ERR_CUDA;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(units * plan.n_cta), 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = plan.n_cta;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, ssd_unit_kernel<TIn, kAligned, kGreedy>, a);
+  return e == cudaSuccess ? SSD_OK : SSD_ERR_CUDA;
+}
+
+static ssd_status launch_units(const UnitArgs& a, int dtype, bool aligned, const Plan& plan, long long units,
+                               cudaStream_t stream) {
+  const bool greedy = a.T == 0.f;
+  if (dtype == SSD_DTYPE_BF16) {
+    if (aligned)
+      return greedy ? launch_units_t<uint16_t, true, true>(a, plan, units, stream)
+                    : launch_units_t<uint16_t, true, false>(a, plan, units, stream);
+    return greedy ? launch_units_t<uint16_t, false, true>(a, plan, units, stream)
+                  : launch_units_t<uint16_t, false, false>(a, plan, units, stream);
+  }
+  if (aligned)
+    return greedy ? launch_units_t<float, true, true>(a, plan, units, stream)
+                  : launch_units_t<float, true, false>(a, plan, units, stream);
+  return greedy ? launch_units_t<float, false, true>(a, plan, units, stream)
+                : launch_units_t<float, false, false>(a, plan, units, stream);
+}
+
+static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+}  // namespace ssd
+
+using namespace ssd;
+
+extern "C" {
+
+const char* ssd_version(void) { return "libssd 0.1 (sm_100a)"; }
+
+const char* ssd_status_string(ssd_status s) {
+  switch (s) {
+    case SSD_OK: return "ok";
+    case SSD_ERR_INVALID_ARG: return "invalid argument";
+    case SSD_ERR_DTYPE: return "unsupported dtype";
+    case SSD_ERR_ALIGNMENT: return "misaligned pointer";
+    case SSD_ERR_WORKSPACE: return "workspace missing or too small";
+    case SSD_ERR_CUDA: return "CUDA launch failed";
+    case SSD_ERR_TIMEOUT: return "device wait timed out";
+    case SSD_ERR_UNSUPPORTED: return "vocabulary too large for this build";
+  }
+  return "unknown status";
+}
+
+size_t ssd_workspace_bytes(int B, int K, int V, int dtype) {
+  (void)V;
+  (void)dtype;
+  if (B < 0 || K < 1 || K > SSD_MAX_K) return 0;
+  return ws_layout(B, K).total;
+}
+
+ssd_status ssd_read_device_error(void* workspace, int B, int K, void* stream, int32_t* out) {
+  if (!workspace || !out || B < 0 || K < 1 || K > SSD_MAX_K) return SSD_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int32_t* word = reinterpret_cast<int32_t*>(static_cast<char*>(workspace) + ws_layout(B, K).error);
+  int32_t v = 0;
+  if (cudaMemcpyAsync(&v, word, sizeof(v), cudaMemcpyDeviceToHost, st) != cudaSuccess) return SSD_ERR_CUDA;
+  if (cudaMemsetAsync(word, 0, sizeof(v), st) != cudaSuccess) return SSD_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return SSD_ERR_CUDA;
+  *out = v ? SSD_ERR_TIMEOUT : SSD_OK;
+  return SSD_OK;
+}
+
+ssd_status ssd_fanout_plan(const float* alpha, int B, int K, int budget, int mode, int32_t* F, void* stream) {
+  if (B < 0 || K < 1 || K > SSD_MAX_K || budget < 0 || budget > SSD_MAX_BUDGET) return SSD_ERR_INVALID_ARG;
+  if (mode != SSD_FANOUT_GEOMETRIC && mode != SSD_FANOUT_UNIFORM) return SSD_ERR_INVALID_ARG;
+  if (B == 0) return SSD_OK;
+  if (!F || (mode == SSD_FANOUT_GEOMETRIC && !alpha)) return SSD_ERR_INVALID_ARG;
+  fanout_kernel<<<(B + 127) / 128, 128, 0, static_cast<cudaStream_t>(stream)>>>(alpha, B, K, budget, mode, F);
+  return cudaGetLastError() == cudaSuccess ? SSD_OK : SSD_ERR_CUDA;
+}
+
+ssd_status ssd_cache_build(const int32_t* F, const int32_t* topf_tokens, const int32_t* guess_K, int B, int K,
+                           int budget, int32_t* offsets, int32_t* tokens, void* stream) {
+  if (B < 0 || K < 1 || K > SSD_MAX_K || budget < 0 || budget > SSD_MAX_BUDGET) return SSD_ERR_INVALID_ARG;
+  if (B == 0) return SSD_OK;
+  if (!F || !topf_tokens || !offsets || !tokens) return SSD_ERR_INVALID_ARG;
+  cache_build_kernel<<<B, 128, 0, static_cast<cudaStream_t>(stream)>>>(F, topf_tokens, guess_K, K, budget, offsets,
+                                                                      tokens);
+  return cudaGetLastError() == cudaSuccess ? SSD_OK : SSD_ERR_CUDA;
+}
+
+ssd_status ssd_cache_lookup(const int32_t* offsets, const int32_t* tokens, int B, int K, int budget,
+                            const int32_t* k, const int32_t* bonus, const int32_t* payload, uint64_t fallback_seed,
+                            int V, uint8_t* hit, int32_t* slot, int32_t* next_tokens, void* stream) {
+  if (B < 0 || K < 1 || K > SSD_MAX_K || budget < 0 || V < 1) return SSD_ERR_INVALID_ARG;
+  if (B == 0) return SSD_OK;
+  if (!offsets || !tokens || !k || !bonus || !hit || !slot || !next_tokens) return SSD_ERR_INVALID_ARG;
+  cache_lookup_kernel<<<(B + 127) / 128, 128, 0, static_cast<cudaStream_t>(stream)>>>(
+      offsets, tokens, B, K, budget, k, bonus, payload, fallback_seed, V, hit, slot, next_tokens);
+  return cudaGetLastError() == cudaSuccess ? SSD_OK : SSD_ERR_CUDA;
+}
+
+ssd_status ssd_verify(const void* target_logits, const void* draft_logits, const void* draft_next, int dtype,
+                      int B, int K, int V, const int32_t* draft_tokens, const float* uniforms, float T,
+                      const int32_t* F, const float* alpha, int fanout_mode, float C, int budget,
+                      int32_t* n_accepted, int32_t* bonus,
+                      int32_t* out_tokens, float* accept_prob, float* residual_mass, const ssd_cache* cache,
+                      int32_t* status, void* workspace, size_t ws_bytes, void* stream) {
+  if (dtype != SSD_DTYPE_BF16 && dtype != SSD_DTYPE_FP32) return SSD_ERR_DTYPE;
+  if (B < 0 || K < 1 || K > SSD_MAX_K || V < 1) return SSD_ERR_INVALID_ARG;
+  if (!(T >= 0.f) || isinf(T)) return SSD_ERR_INVALID_ARG;
+  const bool has_plan = F != nullptr || alpha != nullptr;
+  if (has_plan && (!(C > 0.f && C <= 1.f) || budget < 0 || budget > SSD_MAX_BUDGET || budget > V))
+    return SSD_ERR_INVALID_ARG;
+  if (!F && alpha && fanout_mode != SSD_FANOUT_GEOMETRIC && fanout_mode != SSD_FANOUT_UNIFORM)
+    return SSD_ERR_INVALID_ARG;
+  if (cache && (!has_plan || !cache->offsets || !cache->tokens || !cache->hit || !cache->slot || !cache->next_tokens))
+    return SSD_ERR_INVALID_ARG;
+  if (B == 0) return SSD_OK;
+  if (!target_logits || !draft_logits || !draft_tokens || !uniforms || !n_accepted || !bonus || !out_tokens ||
+      !accept_prob || !residual_mass || !status)
+    return SSD_ERR_INVALID_ARG;
+  if (!aligned16(target_logits) || !aligned16(draft_logits) || (draft_next && !aligned16(draft_next)))
+    return SSD_ERR_ALIGNMENT;
+  if (!workspace || ws_bytes < ws_layout(B, K).total) return SSD_ERR_WORKSPACE;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return SSD_ERR_ALIGNMENT;
+  const int esize = dtype == SSD_DTYPE_BF16 ? 2 : 4;
+  const long long units = static_cast<long long>(B) * (K + 1);
+  Plan plan;
+  const ssd_status ps = make_plan(V, 2, esize, units, &plan);
+  if (ps != SSD_OK) return ps;
+  if (units * plan.n_cta > 0x7FFFFFFFLL) return SSD_ERR_INVALID_ARG;
+  UnitArgs a = {};
+  a.target = target_logits;
+  a.draft = draft_logits;
+  a.draft_next = draft_next;
+  a.tokens = draft_tokens;
+  a.uniforms = uniforms;
+  a.F = F;
+  a.alpha = F ? nullptr : alpha;
+  a.fanout_mode = fanout_mode;
+  a.B = B; a.K = K; a.V = V; a.budget = budget; a.mode = kModeVerify;
+  a.n_cta = plan.n_cta; a.chunk = plan.chunk; a.units_per_row = K + 1;
+  a.T = T; a.C = has_plan ? C : 1.f;
+  a.n_accepted = n_accepted; a.bonus = bonus; a.out_tokens = out_tokens; a.accept_prob = accept_prob;
+  a.residual_mass = residual_mass; a.status = status;
+  if (cache) {
+    a.c_offsets = cache->offsets; a.c_tokens = cache->tokens; a.c_payload = cache->payload;
+    a.c_hit = cache->hit; a.c_slot = cache->slot; a.c_next = cache->next_tokens;
+    a.fallback_seed = cache->fallback_seed;
+  }
+  bind_workspace(a, workspace, B, K);
+  const int VE = 16 / esize;
+  return launch_units(a, dtype, V % VE == 0, plan, units, static_cast<cudaStream_t>(stream));
+}
+
+ssd_status ssd_saguaro_reweight(const void* draft_logits, int dtype, int B, int K, int V, float T, const int32_t* F,
+                                float C, int budget, const void* guess_logits, int64_t guess_row_stride,
+                                const float* u_draft, int32_t* topf_tokens, int32_t* offsets, float* Z,
+                                float* q_lse, int32_t* draft_tokens_out, int32_t* status, void* workspace,
+                                size_t ws_bytes, void* stream) {
+  if (dtype != SSD_DTYPE_BF16 && dtype != SSD_DTYPE_FP32) return SSD_ERR_DTYPE;
+  if (B < 0 || K < 1 || K > SSD_MAX_K || V < 1) return SSD_ERR_INVALID_ARG;
+  if (!(T >= 0.f) || isinf(T) || !(C > 0.f && C <= 1.f)) return SSD_ERR_INVALID_ARG;
+  if (budget < 0 || budget > SSD_MAX_BUDGET || budget > V) return SSD_ERR_INVALID_ARG;
+  if (draft_tokens_out && !u_draft) return SSD_ERR_INVALID_ARG;
+  if (guess_logits && guess_row_stride < V) return SSD_ERR_INVALID_ARG;
+  if (B == 0) return SSD_OK;
+  if (!draft_logits || !F || !topf_tokens || !offsets || !Z || !q_lse || !status) return SSD_ERR_INVALID_ARG;
+  if (!aligned16(draft_logits) || (guess_logits && !aligned16(guess_logits))) return SSD_ERR_ALIGNMENT;
+  if (!workspace || ws_bytes < ws_layout(B, K).total) return SSD_ERR_WORKSPACE;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return SSD_ERR_ALIGNMENT;
+  const int esize = dtype == SSD_DTYPE_BF16 ? 2 : 4;
+  const int per_row = K + (guess_logits ? 1 : 0);
+  const long long units = static_cast<long long>(B) * per_row;
+  Plan plan;
+  const ssd_status ps = make_plan(V, 1, esize, units, &plan);
+  if (ps != SSD_OK) return ps;
+  if (units * plan.n_cta > 0x7FFFFFFFLL) return SSD_ERR_INVALID_ARG;
+  UnitArgs a = {};
+  a.draft = draft_logits;
+  a.guess = guess_logits;
+  a.guess_stride = guess_row_stride;
+  a.uniforms = u_draft;
+  a.F = F;
+  a.B = B; a.K = K; a.V = V; a.budget = budget; a.mode = kModeReweight;
+  a.n_cta = plan.n_cta; a.chunk = plan.chunk; a.units_per_row = per_row;
+  a.T = T; a.C = C;
+  a.status = status;
+  a.topf_tokens = topf_tokens; a.offsets = offsets; a.Z = Z; a.q_lse = q_lse; a.draft_tokens = draft_tokens_out;
+  bind_workspace(a, workspace, B, K);
+  const int VE = 16 / esize;
+  const bool aligned = V % VE == 0 && (!guess_logits || guess_row_stride % VE == 0);
+  return launch_units(a, dtype, aligned, plan, units, static_cast<cudaStream_t>(stream));
+}
+
+}  // extern "C"

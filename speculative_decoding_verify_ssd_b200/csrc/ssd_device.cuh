@@ -1,0 +1,202 @@
+// ssd_device.cuh -- device-side building blocks of libssd (sm_100a only).
+//
+// Bulk global->shared copies completed on an mbarrier, bounded waits, the
+// fast exp2, bf16 unpacking, order-preserving integer keys for logits, and
+// Philox4x32-10 (Salmon, Moraes, Dror, Shaw, "Parallel Random Numbers: As
+// Easy as 1, 2, 3", SC'11, section 4).
+#pragma once
+
+#include <cooperative_groups.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace ssd {
+
+namespace cg = cooperative_groups;
+
+constexpr float kLog2e = 1.4426950408889634f;
+
+// ---------------------------------------------------------------------------
+// Shared-memory addresses, mbarrier and the bulk copy engine.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count) : "memory");
+}
+
+// Make the initialised barrier visible to the async (bulk copy) proxy.
+__device__ __forceinline__ void mbar_init_fence() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile(
+      "{\n\t.reg .b64 st;\n\t"
+      "mbarrier.arrive.expect_tx.shared::cta.b64 st, [%0], %1;\n\t}" ::"r"(smem_addr(bar)),
+      "r"(bytes)
+      : "memory");
+}
+
+// One poll; the thread may be suspended (up to `hint_ns`) until the phase
+// completes, so a waiting warp costs almost no issue slots.
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
+  uint32_t done;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(done)
+      : "r"(smem_addr(bar)), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return done != 0;
+}
+
+// Bounded wait: polls, and between unsuccessful polls puts the warp to sleep
+// (exponential backoff up to ~0.5 us) so that a waiting warp does not take
+// issue slots from co-resident CTAs.  Gives up after `max_polls` polls and
+// returns false.
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, uint32_t max_polls) {
+  uint32_t sleep_ns = 32;
+  for (uint32_t i = 0; i < max_polls; ++i) {
+    if (mbar_try_wait(bar, parity, 0u)) return true;
+    __nanosleep(sleep_ns);
+    if (sleep_ns < 512) sleep_ns <<= 1;
+  }
+  return false;
+}
+
+// 1-D bulk copy global -> this CTA's shared memory (no multicast).  Both
+// addresses 16-byte aligned, bytes a multiple of 16.
+__device__ __forceinline__ void bulk_copy_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_addr(dst)),
+      "l"(static_cast<uint64_t>(__cvta_generic_to_global(src))), "r"(bytes), "r"(smem_addr(bar))
+      : "memory");
+}
+
+// Split cluster barrier (all threads of every CTA of the cluster): arrive
+// with release semantics, wait with acquire semantics.  Every thread
+// alternates arrive and wait.
+__device__ __forceinline__ void cluster_arrive() {
+  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait() {
+  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_sync_all() {
+  cluster_arrive();
+  cluster_wait();
+}
+
+// ---------------------------------------------------------------------------
+// Arithmetic helpers.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// max with NaN propagation (a NaN anywhere makes the result NaN).
+__device__ __forceinline__ float fmax_nan(float a, float b) {
+  float d;
+  asm("max.NaN.f32 %0, %1, %2;" : "=f"(d) : "f"(a), "f"(b));
+  return d;
+}
+
+__device__ __forceinline__ uint32_t bf16x2_max_nan(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("max.NaN.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+// Order-preserving key of a float logit: larger logit -> larger key; -0 and
+// +0 map to the same key so that they tie (and the lower token id wins).
+__device__ __forceinline__ uint32_t ord_key(float f) {
+  uint32_t u = __float_as_uint(f);
+  if ((u & 0x7FFFFFFFu) == 0u) u = 0u;
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// Composite ranking key: logit descending, then token id ascending.
+__device__ __forceinline__ unsigned long long rank_key(float f, int idx) {
+  return (static_cast<unsigned long long>(ord_key(f)) << 32) |
+         static_cast<unsigned long long>(0xFFFFFFFFu - static_cast<uint32_t>(idx));
+}
+
+// ---------------------------------------------------------------------------
+// Philox4x32-10 (Salmon et al., SC'11): ten rounds, key bumped by the Weyl
+// constants after each round.
+// ---------------------------------------------------------------------------
+struct U4 {
+  uint32_t x, y, z, w;
+};
+
+__device__ __forceinline__ U4 philox4x32_10(U4 c, uint32_t k0, uint32_t k1) {
+#pragma unroll
+  for (int r = 0; r < 10; ++r) {
+    const uint32_t lo0 = 0xD2511F53u * c.x;
+    const uint32_t hi0 = __umulhi(0xD2511F53u, c.x);
+    const uint32_t lo1 = 0xCD9E8D57u * c.z;
+    const uint32_t hi1 = __umulhi(0xCD9E8D57u, c.z);
+    c = U4{hi1 ^ c.y ^ k0, lo1, hi0 ^ c.w ^ k1, lo0};
+    k0 += 0x9E3779B9u;
+    k1 += 0xBB67AE85u;
+  }
+  return c;
+}
+
+// Fallback speculator token i of row b: floor(x * V / 2^32), x = word 0 at
+// counter (b, i, 2, 0), key = seed.
+__device__ __forceinline__ int32_t fallback_token(unsigned long long seed, int b, int i, int V) {
+  const U4 o = philox4x32_10(U4{static_cast<uint32_t>(b), static_cast<uint32_t>(i), 2u, 0u},
+                             static_cast<uint32_t>(seed), static_cast<uint32_t>(seed >> 32));
+  return static_cast<int32_t>((static_cast<unsigned long long>(o.x) * static_cast<uint32_t>(V)) >> 32);
+}
+
+// ---------------------------------------------------------------------------
+// Warp reductions.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
+  return v;
+}
+
+__device__ __forceinline__ float warp_max_nan(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmax_nan(v, __shfl_xor_sync(0xFFFFFFFFu, v, o));
+  return v;
+}
+
+// The F-th largest of n order keys held by one warp (keys[i] for i = lane,
+// lane + 32, ...): bitwise search for the largest t with #{key >= t} >= F,
+// high bit first.  `bits` = number of significant high bits of the keys.
+template <int kPerLane>
+__device__ __forceinline__ uint32_t warp_kth_largest(const uint32_t (&keys)[kPerLane], int F, int bits) {
+  uint32_t prefix = 0u;
+  for (int bit = 31; bit >= 32 - bits; --bit) {
+    const uint32_t cand = prefix | (1u << bit);
+    int c = 0;
+#pragma unroll
+    for (int i = 0; i < kPerLane; ++i) c += keys[i] >= cand;
+    c = __reduce_add_sync(0xFFFFFFFFu, c);
+    if (c >= F) prefix = cand;
+  }
+  return prefix;
+}
+
+// Inverse of ord_key.
+__device__ __forceinline__ float key_to_float(uint32_t k) {
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
+}
+
+}  // namespace ssd
