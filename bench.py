@@ -165,7 +165,7 @@ def run_ssd(args, rank, world, local_rank):
         sets.append(dict(t=t, d=d, alpha=alpha, u=u, tok=rw.draft_tokens))
         del g
     torch.cuda.synchronize()
-    ws = ssd.Workspace(w.B, w.K, dev)
+    ws = ssd.Workspace(w.B, w.K, dev, w.V, ssd.DTYPE_BF16 if w.dtype == "bf16" else ssd.DTYPE_FP32)
     outs = [ssd.alloc_verify_result(w.B, w.K, w.budget, dev, True) for _ in range(n_copies)]
 
     def step(i):

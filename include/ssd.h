@@ -188,18 +188,20 @@ ssd_status ssd_cache_lookup(const int32_t* offsets, const int32_t* tokens, int B
                             const int32_t* payload, uint64_t fallback_seed, int V,
                             uint8_t* hit, int32_t* slot, int32_t* next_tokens, void* stream);
 
-/* Workspace size in bytes for ssd_verify / ssd_saguaro_reweight at (B, K).
- * The workspace holds per-(row, position) results, then per-row arrival
- * counters and skip hints, then one device error word.  It must be 256-byte
- * aligned and zero-filled before its first use; each completed call leaves
- * the counters and hints zero again, so it can be reused by the next call on
- * the same stream (calls that overlap on the GPU must not share one). */
+/* Workspace size in bytes for ssd_verify / ssd_saguaro_reweight at
+ * (B, K, V, dtype).  The workspace holds per-slice and per-(row, position)
+ * partial results, per-row states, then arrival counters and one device error
+ * word.  It must be 256-byte aligned and zero-filled before its first use;
+ * each completed call leaves the counters zero again, so it can be reused by
+ * the next call on the same stream (calls that overlap on the GPU must not
+ * share one).  0 for invalid sizes. */
 size_t ssd_workspace_bytes(int B, int K, int V, int dtype);
 
-/* Reads and clears the device error word of a workspace laid out for (B, K),
- * synchronising `stream`: *out = SSD_OK, or SSD_ERR_TIMEOUT when a bounded
- * device wait of an earlier call gave up.  Not for the hot path. */
-ssd_status ssd_read_device_error(void* workspace, int B, int K, void* stream, int32_t* out);
+/* Reads and clears the device error word of a workspace laid out for
+ * (B, K, V, dtype), synchronising `stream`: *out = SSD_OK, or SSD_ERR_TIMEOUT
+ * when a bounded device wait of an earlier call gave up.  Not for the hot path. */
+ssd_status ssd_read_device_error(void* workspace, int B, int K, int V, int dtype, void* stream,
+                                 int32_t* out);
 
 const char* ssd_status_string(ssd_status s);
 const char* ssd_version(void);

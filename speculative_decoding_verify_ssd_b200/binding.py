@@ -70,7 +70,7 @@ def load(build_if_missing: bool = True):
     L.ssd_workspace_bytes.restype = sz
     L.ssd_workspace_bytes.argtypes = [i32, i32, i32, i32]
     L.ssd_read_device_error.restype = i32
-    L.ssd_read_device_error.argtypes = [vp, i32, i32, vp, C.POINTER(C.c_int32)]
+    L.ssd_read_device_error.argtypes = [vp, i32, i32, i32, i32, vp, C.POINTER(C.c_int32)]
     L.ssd_fanout_plan.restype = i32
     L.ssd_fanout_plan.argtypes = [vp, i32, i32, i32, i32, vp, vp]
     L.ssd_saguaro_reweight.restype = i32
@@ -135,12 +135,13 @@ def workspace_bytes(B: int, K: int, V: int = 0, dtype: int = DTYPE_BF16) -> int:
 
 
 class Workspace:
-    """Caller-owned, zero-filled device workspace, reusable across calls on
-    one stream (every completed call leaves it zero-filled)."""
+    """Caller-owned, zero-filled device workspace for (B, K, V, dtype),
+    reusable across calls on one stream (each completed call leaves its
+    counters zero)."""
 
-    def __init__(self, B: int, K: int, device):
-        self.B, self.K = B, K
-        self.nbytes = workspace_bytes(B, K)
+    def __init__(self, B: int, K: int, device, V: int = 262144, dtype: int = DTYPE_BF16):
+        self.B, self.K, self.V, self.dtype = B, K, V, dtype
+        self.nbytes = workspace_bytes(B, K, V, dtype)
         self.buf = torch.zeros(self.nbytes + 256, dtype=torch.uint8, device=device)
         off = (-self.buf.data_ptr()) % 256
         self.view = self.buf[off:off + self.nbytes]
@@ -150,7 +151,8 @@ class Workspace:
 
     def device_error(self, stream=None) -> int:
         out = C.c_int32(0)
-        _check(load().ssd_read_device_error(self.ptr(), self.B, self.K, _stream(stream), C.byref(out)),
+        _check(load().ssd_read_device_error(self.ptr(), self.B, self.K, self.V, self.dtype, _stream(stream),
+                                            C.byref(out)),
                "ssd_read_device_error")
         return out.value
 
@@ -227,7 +229,7 @@ def ssd_verify(target: torch.Tensor, draft: torch.Tensor, draft_tokens: torch.Te
     if cache and F is None and alpha is None:
         raise ValueError("a cache needs a fan-out plan (F or alpha)")
     if workspace is None:
-        workspace = Workspace(B, K, dev)
+        workspace = Workspace(B, K, dev, V, dt)
     if out is None:
         out = alloc_verify_result(B, K, budget, dev, cache)
     cstruct = None
@@ -292,7 +294,7 @@ def ssd_saguaro_reweight(draft: torch.Tensor, T: float, F: torch.Tensor, C_coef:
             raise ValueError("guess rows must match the draft dtype and device")
         stride = int(guess_row_stride if guess_row_stride is not None else guess.stride(0))
     if workspace is None:
-        workspace = Workspace(B, K, dev)
+        workspace = Workspace(B, K, dev, V, dt)
     i32 = dict(dtype=torch.int32, device=dev)
     r = ReweightResult(topf_tokens=torch.full((B, max(budget, 1)), -2, **i32),
                        offsets=torch.empty((B, K + 2), **i32),

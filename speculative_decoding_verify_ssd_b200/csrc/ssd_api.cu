@@ -1,6 +1,7 @@
 // ssd_api.cu -- host side of libssd: argument checks, launch planning and the
 // extern "C" entry points declared in include/ssd.h, plus the three small
-// kernels (fan-out plan, cache build, cache lookup).
+// kernels (fan-out plan, cache build, cache lookup).  The two vocab-wide
+// kernels live in ssd_kernels.cuh.
 #include <cuda_runtime.h>
 #include <math.h>
 #include <stdint.h>
@@ -11,7 +12,7 @@
 
 #include "../../include/ssd.h"
 #include "ssd_device.cuh"
-#include "ssd_unit_kernel.cuh"
+#include "ssd_kernels.cuh"
 
 namespace ssd {
 
@@ -101,14 +102,13 @@ __global__ void cache_lookup_kernel(const int32_t* __restrict__ offsets, const i
 // Launch planning.
 // ---------------------------------------------------------------------------
 #ifndef SSD_CTA_BYTES
-#define SSD_CTA_BYTES 65536   // logits streamed per CTA per unit (all rows of the unit)
+#define SSD_CTA_BYTES 65536   // logits streamed per CTA (all rows of a unit slice)
 #endif
 constexpr long long kCtaBytes = SSD_CTA_BYTES;
 constexpr int kMinChunk = 1024;  // do not split a row finer than this
 
 struct Plan {
-  int n_cta, chunk;
-  size_t smem;  // bulk-copy ring (aligned rows only)
+  int n_slices, chunk;
 };
 
 static int sm_count() {
@@ -117,113 +117,132 @@ static int sm_count() {
   return n > 0 ? n : 148;
 }
 
-// Cluster size and slice length for one unit of `rows` logit rows of length V.
+// Slices per logit row and the slice length, for units of `rows` rows of length V.
 static ssd_status make_plan(int V, int rows, int esize, long long units, Plan* p) {
   const int VE = 16 / esize;
   const long long max_chunk = static_cast<long long>(kMaxChunks) * kChunkVecs * VE;
-  long long n_cta = (static_cast<long long>(rows) * V * esize + kCtaBytes - 1) / kCtaBytes;
-  // Enough CTAs to fill the machine, if the rows are long enough.
+  long long ns = (static_cast<long long>(rows) * V * esize + kCtaBytes - 1) / kCtaBytes;
+  // enough CTAs to fill the machine, if the rows are long enough
   const long long want = (static_cast<long long>(kMinBlocks) * sm_count() + units - 1) / (units > 0 ? units : 1);
   const long long by_len = (V + kMinChunk - 1) / kMinChunk;
   long long extra = want < by_len ? want : by_len;
   if (extra > 8) extra = 8;
-  if (n_cta < extra) n_cta = extra;
-  if (n_cta < 1) n_cta = 1;
-  long long chunk = (V + n_cta - 1) / n_cta;
+  if (ns < extra) ns = extra;
+  if (ns < 1) ns = 1;
+  long long chunk = (V + ns - 1) / ns;
   chunk = (chunk + VE - 1) / VE * VE;
   if (chunk > max_chunk) {
-    n_cta = (V + max_chunk - 1) / max_chunk;
-    chunk = (V + n_cta - 1) / n_cta;
+    ns = (V + max_chunk - 1) / max_chunk;
+    chunk = (V + ns - 1) / ns;
     chunk = (chunk + VE - 1) / VE * VE;
   }
-  n_cta = (V + chunk - 1) / chunk;
-  if (n_cta > kMaxCluster) return SSD_ERR_UNSUPPORTED;
-  p->n_cta = static_cast<int>(n_cta);
+  ns = (V + chunk - 1) / chunk;
+  if (ns > kMaxSlices) return SSD_ERR_UNSUPPORTED;
+  p->n_slices = static_cast<int>(ns);
   p->chunk = static_cast<int>(chunk);
-  p->smem = static_cast<size_t>(kStages) * (rows > 1 ? 2 : 1) * kChunkVecs * 16;
   return SSD_OK;
 }
 
 static std::mutex g_attr_mu;
 static std::map<std::tuple<const void*, int>, int> g_attr_done;
 
-static cudaError_t prepare_kernel(const void* fn, size_t smem) {
+static cudaError_t prepare_kernel(const void* fn) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   std::lock_guard<std::mutex> lock(g_attr_mu);
   auto key = std::make_tuple(fn, dev);
-  auto it = g_attr_done.find(key);
-  if (it != g_attr_done.end() && it->second >= static_cast<int>(smem)) return cudaSuccess;
-  // clusters of up to 16 CTAs; the bulk-copy ring in dynamic shared memory
-  e = cudaFuncSetAttribute(fn, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+  if (g_attr_done.count(key)) return cudaSuccess;
+  e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kRingBytes));
   if (e != cudaSuccess) return e;
-  e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-  if (e != cudaSuccess) return e;
-  g_attr_done[key] = static_cast<int>(smem);
+  g_attr_done[key] = 1;
   return cudaSuccess;
 }
 
+// Workspace: slice partials, unit states, draw partials, row states, then the
+// counters (zero between calls) and the error word.
 struct WsLayout {
-  size_t units, counters, first_rej, error, total;
+  size_t parts, ustate, dparts, rstate, arrive1, row_arrive, draw_arrive, row_arrive2, error, total;
+  int n_slices;
 };
 
-static WsLayout ws_layout(int B, int K) {
+static int plan_slices(int B, int K, int V, int dtype) {
+  const int esize = dtype == SSD_DTYPE_FP32 ? 4 : 2;
+  Plan p2, p1;
+  const long long units = static_cast<long long>(B) * (K + 1);
+  int ns = 1;
+  if (make_plan(V, 2, esize, units, &p2) == SSD_OK) ns = p2.n_slices;
+  if (make_plan(V, 1, esize, units, &p1) == SSD_OK) ns = ns > p1.n_slices ? ns : p1.n_slices;
+  return ns;
+}
+
+static size_t up256(size_t x) { return (x + 255) / 256 * 256; }
+
+static WsLayout ws_layout(int B, int K, int V, int dtype) {
   WsLayout w;
   const size_t nb = static_cast<size_t>(B > 0 ? B : 0);
-  w.units = 0;
-  w.counters = w.units + nb * static_cast<size_t>(K + 1) * sizeof(UnitRes);
-  w.first_rej = w.counters + nb * sizeof(int32_t);
-  w.error = w.first_rej + nb * sizeof(int32_t);
-  w.total = (w.error + sizeof(int32_t) + 255) / 256 * 256;
+  const size_t units = nb * static_cast<size_t>(K + 1);
+  const size_t ns = static_cast<size_t>(plan_slices(B, K, V, dtype));
+  w.n_slices = static_cast<int>(ns);
+  size_t off = 0;
+  w.parts = off;       off = up256(off + units * ns * sizeof(SlicePart));
+  w.ustate = off;      off = up256(off + units * sizeof(UnitState));
+  w.dparts = off;      off = up256(off + nb * static_cast<size_t>(K) * ns * sizeof(DrawPart));
+  w.rstate = off;      off = up256(off + nb * sizeof(RowState));
+  w.arrive1 = off;     off += units * sizeof(int32_t);
+  w.row_arrive = off;  off += nb * sizeof(int32_t);
+  w.draw_arrive = off; off += nb * static_cast<size_t>(K) * sizeof(int32_t);
+  w.row_arrive2 = off; off += nb * sizeof(int32_t);
+  w.error = off;       off += sizeof(int32_t);
+  w.total = up256(off);
   return w;
 }
 
-static void bind_workspace(UnitArgs& a, void* ws, int B, int K) {
-  const WsLayout w = ws_layout(B, K);
+static void bind_workspace(Args& a, void* ws, const WsLayout& w) {
   char* base = static_cast<char*>(ws);
-  a.units = reinterpret_cast<UnitRes*>(base + w.units);
-  a.counters = reinterpret_cast<int32_t*>(base + w.counters);
-  a.first_rej = reinterpret_cast<int32_t*>(base + w.first_rej);
+  a.parts = reinterpret_cast<SlicePart*>(base + w.parts);
+  a.ustate = reinterpret_cast<UnitState*>(base + w.ustate);
+  a.dparts = reinterpret_cast<DrawPart*>(base + w.dparts);
+  a.rstate = reinterpret_cast<RowState*>(base + w.rstate);
+  a.arrive1 = reinterpret_cast<int32_t*>(base + w.arrive1);
+  a.row_arrive = reinterpret_cast<int32_t*>(base + w.row_arrive);
+  a.draw_arrive = reinterpret_cast<int32_t*>(base + w.draw_arrive);
+  a.row_arrive2 = reinterpret_cast<int32_t*>(base + w.row_arrive2);
   a.error = reinterpret_cast<int32_t*>(base + w.error);
 }
 
 template <typename TIn, bool kAligned, bool kGreedy>
-static ssd_status launch_units_t(const UnitArgs& a, const Plan& plan, long long units, cudaStream_t stream) {
-  const void* fn = reinterpret_cast<const void*>(&ssd_unit_kernel<TIn, kAligned, kGreedy>);
-  const size_t smem = kAligned ? plan.smem : 0;
-  if (prepare_kernel(fn, smem) != cudaSuccess) return SSD_ERR_CUDA;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(units * plan.n_cta), 1, 1);
-  cfg.blockDim = dim3(kThreads, 1, 1);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = plan.n_cta;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  const cudaError_t e = cudaLaunchKernelEx(&cfg, ssd_unit_kernel<TIn, kAligned, kGreedy>, a);
-  return e == cudaSuccess ? SSD_OK : SSD_ERR_CUDA;
+static ssd_status launch_t(const Args& a, long long units, long long draw_units, cudaStream_t stream) {
+  const void* f1 = reinterpret_cast<const void*>(&ssd_stats_kernel<TIn, kAligned, kGreedy>);
+  const void* f2 = reinterpret_cast<const void*>(&ssd_draw_kernel<TIn, kAligned, kGreedy>);
+  if (prepare_kernel(f1) != cudaSuccess || prepare_kernel(f2) != cudaSuccess) return SSD_ERR_CUDA;
+  const size_t smem = kAligned ? kRingBytes : 0;
+  ssd_stats_kernel<TIn, kAligned, kGreedy>
+      <<<static_cast<unsigned>(units * a.n_slices), kThreads, smem, stream>>>(a);
+  if (cudaGetLastError() != cudaSuccess) return SSD_ERR_CUDA;
+  if (draw_units > 0) {
+    ssd_draw_kernel<TIn, kAligned, kGreedy>
+        <<<static_cast<unsigned>(draw_units * a.n_slices), kThreads, smem, stream>>>(a);
+    if (cudaGetLastError() != cudaSuccess) return SSD_ERR_CUDA;
+  }
+  return SSD_OK;
 }
 
-static ssd_status launch_units(const UnitArgs& a, int dtype, bool aligned, const Plan& plan, long long units,
-                               cudaStream_t stream) {
+static ssd_status launch(const Args& a, int dtype, bool aligned, long long units, long long draw_units,
+                         cudaStream_t stream) {
   const bool greedy = a.T == 0.f;
   if (dtype == SSD_DTYPE_BF16) {
     if (aligned)
-      return greedy ? launch_units_t<uint16_t, true, true>(a, plan, units, stream)
-                    : launch_units_t<uint16_t, true, false>(a, plan, units, stream);
-    return greedy ? launch_units_t<uint16_t, false, true>(a, plan, units, stream)
-                  : launch_units_t<uint16_t, false, false>(a, plan, units, stream);
+      return greedy ? launch_t<uint16_t, true, true>(a, units, draw_units, stream)
+                    : launch_t<uint16_t, true, false>(a, units, draw_units, stream);
+    return greedy ? launch_t<uint16_t, false, true>(a, units, draw_units, stream)
+                  : launch_t<uint16_t, false, false>(a, units, draw_units, stream);
   }
   if (aligned)
-    return greedy ? launch_units_t<float, true, true>(a, plan, units, stream)
-                  : launch_units_t<float, true, false>(a, plan, units, stream);
-  return greedy ? launch_units_t<float, false, true>(a, plan, units, stream)
-                : launch_units_t<float, false, false>(a, plan, units, stream);
+    return greedy ? launch_t<float, true, true>(a, units, draw_units, stream)
+                  : launch_t<float, true, false>(a, units, draw_units, stream);
+  return greedy ? launch_t<float, false, true>(a, units, draw_units, stream)
+                : launch_t<float, false, false>(a, units, draw_units, stream);
 }
 
 static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -251,16 +270,16 @@ const char* ssd_status_string(ssd_status s) {
 }
 
 size_t ssd_workspace_bytes(int B, int K, int V, int dtype) {
-  (void)V;
-  (void)dtype;
-  if (B < 0 || K < 1 || K > SSD_MAX_K) return 0;
-  return ws_layout(B, K).total;
+  if (B < 0 || K < 1 || K > SSD_MAX_K || V < 1) return 0;
+  if (dtype != SSD_DTYPE_BF16 && dtype != SSD_DTYPE_FP32) return 0;
+  return ws_layout(B, K, V, dtype).total;
 }
 
-ssd_status ssd_read_device_error(void* workspace, int B, int K, void* stream, int32_t* out) {
-  if (!workspace || !out || B < 0 || K < 1 || K > SSD_MAX_K) return SSD_ERR_INVALID_ARG;
+ssd_status ssd_read_device_error(void* workspace, int B, int K, int V, int dtype, void* stream, int32_t* out) {
+  if (!workspace || !out || B < 0 || K < 1 || K > SSD_MAX_K || V < 1) return SSD_ERR_INVALID_ARG;
+  if (dtype != SSD_DTYPE_BF16 && dtype != SSD_DTYPE_FP32) return SSD_ERR_DTYPE;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  int32_t* word = reinterpret_cast<int32_t*>(static_cast<char*>(workspace) + ws_layout(B, K).error);
+  int32_t* word = reinterpret_cast<int32_t*>(static_cast<char*>(workspace) + ws_layout(B, K, V, dtype).error);
   int32_t v = 0;
   if (cudaMemcpyAsync(&v, word, sizeof(v), cudaMemcpyDeviceToHost, st) != cudaSuccess) return SSD_ERR_CUDA;
   if (cudaMemsetAsync(word, 0, sizeof(v), st) != cudaSuccess) return SSD_ERR_CUDA;
@@ -321,15 +340,17 @@ ssd_status ssd_verify(const void* target_logits, const void* draft_logits, const
     return SSD_ERR_INVALID_ARG;
   if (!aligned16(target_logits) || !aligned16(draft_logits) || (draft_next && !aligned16(draft_next)))
     return SSD_ERR_ALIGNMENT;
-  if (!workspace || ws_bytes < ws_layout(B, K).total) return SSD_ERR_WORKSPACE;
+  const WsLayout wl = ws_layout(B, K, V, dtype);
+  if (!workspace || ws_bytes < wl.total) return SSD_ERR_WORKSPACE;
   if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return SSD_ERR_ALIGNMENT;
   const int esize = dtype == SSD_DTYPE_BF16 ? 2 : 4;
   const long long units = static_cast<long long>(B) * (K + 1);
   Plan plan;
   const ssd_status ps = make_plan(V, 2, esize, units, &plan);
   if (ps != SSD_OK) return ps;
-  if (units * plan.n_cta > 0x7FFFFFFFLL) return SSD_ERR_INVALID_ARG;
-  UnitArgs a = {};
+  if (plan.n_slices > wl.n_slices) return SSD_ERR_WORKSPACE;
+  if (units * plan.n_slices > 0x7FFFFFFFLL) return SSD_ERR_INVALID_ARG;
+  Args a = {};
   a.target = target_logits;
   a.draft = draft_logits;
   a.draft_next = draft_next;
@@ -339,7 +360,7 @@ ssd_status ssd_verify(const void* target_logits, const void* draft_logits, const
   a.alpha = F ? nullptr : alpha;
   a.fanout_mode = fanout_mode;
   a.B = B; a.K = K; a.V = V; a.budget = budget; a.mode = kModeVerify;
-  a.n_cta = plan.n_cta; a.chunk = plan.chunk; a.units_per_row = K + 1;
+  a.n_slices = plan.n_slices; a.chunk = plan.chunk; a.units_per_row = K + 1; a.draws = 1;
   a.T = T; a.C = has_plan ? C : 1.f;
   a.n_accepted = n_accepted; a.bonus = bonus; a.out_tokens = out_tokens; a.accept_prob = accept_prob;
   a.residual_mass = residual_mass; a.status = status;
@@ -348,9 +369,9 @@ ssd_status ssd_verify(const void* target_logits, const void* draft_logits, const
     a.c_hit = cache->hit; a.c_slot = cache->slot; a.c_next = cache->next_tokens;
     a.fallback_seed = cache->fallback_seed;
   }
-  bind_workspace(a, workspace, B, K);
+  bind_workspace(a, workspace, wl);
   const int VE = 16 / esize;
-  return launch_units(a, dtype, V % VE == 0, plan, units, static_cast<cudaStream_t>(stream));
+  return launch(a, dtype, V % VE == 0, units, B, static_cast<cudaStream_t>(stream));
 }
 
 ssd_status ssd_saguaro_reweight(const void* draft_logits, int dtype, int B, int K, int V, float T, const int32_t* F,
@@ -367,30 +388,35 @@ ssd_status ssd_saguaro_reweight(const void* draft_logits, int dtype, int B, int 
   if (B == 0) return SSD_OK;
   if (!draft_logits || !F || !topf_tokens || !offsets || !Z || !q_lse || !status) return SSD_ERR_INVALID_ARG;
   if (!aligned16(draft_logits) || (guess_logits && !aligned16(guess_logits))) return SSD_ERR_ALIGNMENT;
-  if (!workspace || ws_bytes < ws_layout(B, K).total) return SSD_ERR_WORKSPACE;
+  const WsLayout wl = ws_layout(B, K, V, dtype);
+  if (!workspace || ws_bytes < wl.total) return SSD_ERR_WORKSPACE;
   if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return SSD_ERR_ALIGNMENT;
   const int esize = dtype == SSD_DTYPE_BF16 ? 2 : 4;
   const int per_row = K + (guess_logits ? 1 : 0);
   const long long units = static_cast<long long>(B) * per_row;
   Plan plan;
-  const ssd_status ps = make_plan(V, 1, esize, units, &plan);
+  const ssd_status ps = make_plan(V, 1, esize, static_cast<long long>(B) * (K + 1), &plan);
   if (ps != SSD_OK) return ps;
-  if (units * plan.n_cta > 0x7FFFFFFFLL) return SSD_ERR_INVALID_ARG;
-  UnitArgs a = {};
+  if (plan.n_slices > wl.n_slices) return SSD_ERR_WORKSPACE;
+  if (units * plan.n_slices > 0x7FFFFFFFLL) return SSD_ERR_INVALID_ARG;
+  Args a = {};
   a.draft = draft_logits;
   a.guess = guess_logits;
   a.guess_stride = guess_row_stride;
   a.uniforms = u_draft;
   a.F = F;
   a.B = B; a.K = K; a.V = V; a.budget = budget; a.mode = kModeReweight;
-  a.n_cta = plan.n_cta; a.chunk = plan.chunk; a.units_per_row = per_row;
+  a.n_slices = plan.n_slices; a.chunk = plan.chunk; a.units_per_row = per_row;
   a.T = T; a.C = C;
   a.status = status;
   a.topf_tokens = topf_tokens; a.offsets = offsets; a.Z = Z; a.q_lse = q_lse; a.draft_tokens = draft_tokens_out;
-  bind_workspace(a, workspace, B, K);
+  bind_workspace(a, workspace, wl);
   const int VE = 16 / esize;
   const bool aligned = V % VE == 0 && (!guess_logits || guess_row_stride % VE == 0);
-  return launch_units(a, dtype, aligned, plan, units, static_cast<cudaStream_t>(stream));
+  const bool draws = u_draft && draft_tokens_out && T > 0.f;
+  a.draws = draws ? 1 : 0;
+  const long long draw_units = draws ? static_cast<long long>(B) * K : 0;
+  return launch(a, dtype, aligned, units, draw_units, static_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"

@@ -1,0 +1,1328 @@
+// ssd_kernels.cuh -- the vocab-wide kernels of libssd.
+//
+// The step runs as two kernels that talk through the caller's workspace:
+//
+// Kernel 1 (stats): one CTA per (unit, slice), unit = (row b, position j).
+//   The CTA streams its slice of the unit's target row p_j and draft row q_j
+//   from HBM exactly once through a ring of 1-D bulk copies into shared
+//   memory (cp.async.bulk completed on mbarriers, no multicast) and keeps per
+//   thread only running softmax state ([ZH] = "Speculative Speculative
+//   Decoding", gist.science Chinese edition, technical summary section 2;
+//   [NL] = the Dutch edition, sections 2 and 3A-3C):
+//     - online max and rescaled sum of exp2 of p_j and q_j (temperature
+//       softmax, one exp per element), or the greedy argmax when T = 0;
+//     - the top two vector maxima of the top-F source row (q_j) and the vector
+//       holding the larger, so the slice's own top-F (which contains the
+//       slice's share of the unit's top-F, [ZH] challenge 2 "top-F tokens")
+//       comes from registers: the F-th largest thread maximum bounds it from
+//       below.
+//   It publishes a small partial and leaves.  The last CTA of a unit to
+//   arrive (a counter, no waiting) merges the partials, selects the exact
+//   top-F by (logit desc, token id asc), forms Q_S and the Saguaro normaliser
+//   Z = 1 - (1 - C) Q_S ([ZH] challenge 2; [NL] 3B), and runs the lossless
+//   accept test a_j = min(1, p_j(d_j) / q'_j(d_j)); the last unit of a row
+//   fixes k*, the first rejected position.  Units are issued in decreasing
+//   position order, so the rows most often needed next are still in L2.
+//
+// Kernel 2 (draw): one CTA per (row, slice) of the single unit each row
+//   draws from: the residual r = max(0, p_k* - q'_k*) (or p_K after full
+//   acceptance, or q' for a draft draw).  Each CTA sums its slice of r per
+//   (ring chunk, warp); the last CTA of the row finds where the cumulative
+//   mass crosses u * R in token order (slice, chunk, warp, then one re-read
+//   vector per lane), draws the bonus token, and finishes the row: outputs,
+//   the cache lookup of (k*, bonus) and the random-token fallback ([ZH]
+//   basic flow steps 3-4 and challenge 3; [NL] 3C).
+#pragma once
+
+#include <limits.h>
+
+#include "../../include/ssd.h"
+#include "ssd_device.cuh"
+
+namespace ssd {
+
+constexpr int kThreads = 256;
+constexpr int kWarps = kThreads / 32;
+constexpr int kMinBlocks = 4;          // CTAs per SM the register budget is set for
+constexpr int kMaxSlices = 16;         // slices per logit row
+constexpr int kStages = 4;             // depth of the bulk-copy ring
+constexpr int kChunkVecs = kThreads;   // 16-byte vectors per row per ring stage
+constexpr int kMaxChunks = 16;         // ring chunks per slice
+constexpr int kCandCap = 256;          // local top-F candidates found by a CTA
+constexpr int kCandSlice = 128;        // candidates a slice publishes
+constexpr int kGatherCap = 1024;       // candidates of a whole unit
+constexpr int kSelCap = 512;           // >= SSD_MAX_BUDGET
+constexpr int kMaxGroups = kThreads;   // thread maxima per CTA
+constexpr uint32_t kMaxPolls = 4000000u;  // x ~0.5 us sleep: about 2 s
+constexpr float kNearTie = 1e-5f;
+constexpr int kFlagTimeout = SSD_ROW_DEVICE_TIMEOUT;
+constexpr size_t kRingBytes = static_cast<size_t>(kStages) * 2 * kChunkVecs * 16;
+
+enum Mode : int { kModeVerify = 0, kModeReweight = 1 };
+enum Draw : int { kDrawNone = 0, kDrawResidual = 1, kDrawP = 2, kDrawQ = 3 };
+
+struct Cand {
+  float x;
+  int32_t idx;
+};
+
+// Kernel 1, one per (unit, slice).
+struct SlicePart {
+  float mP, sP, mQ, sQ;           // running max and exp-sum of the slice
+  int32_t argP, argQ;             // greedy: lowest id of the slice maximum
+  int32_t n_cand, timeout;        // local candidates found; copy timeout
+  Cand cand[kCandSlice];          // sorted local candidates (at most min(n_cand, F))
+};
+
+// Kernel 1, written by the unit's finalizer.
+struct UnitState {
+  float MP, SP, MQ, SQ;           // unit maxima and exp-sums (relative to the maxima)
+  float Z, bx, a, amargin;        // Saguaro normaliser, top-F boundary logit, a_j, |u_j - a_j|
+  int32_t bi, argP, argQ, flags;  // top-F boundary id, greedy argmaxes, SSD_ROW_* bits
+  int32_t rejected, Fj, seg_off;  // u_j >= a_j; the unit's fan-out; its cache segment
+  float dmargin;                  // draft draw: inverse-CDF margin
+};
+
+// Kernel 2, one per (draw unit, slice).
+struct DrawPart {
+  float R, RP;                    // slice mass of the draw's distribution (and of p alone)
+  int32_t timeout, pad;
+  float rs[kMaxChunks][kWarps];   // per (chunk, warp) partial sums, token order
+  float ps[kMaxChunks][kWarps];
+};
+
+struct RowState {
+  int32_t kstar, flags;
+  float amargin;
+  int32_t pad;
+};
+
+struct Args {
+  const void* target;      // [B, K+1, V]
+  const void* draft;       // [B, K, V]
+  const void* draft_next;  // [B, V] or null (verify: source of the full-acceptance guesses)
+  const void* guess;       // reweight: rows for segment K, or null
+  long long guess_stride;
+  const int32_t* tokens;   // [B, K]
+  const float* uniforms;   // [B, K+1] (verify) or u_draft [B, K] (reweight), may be null
+  const int32_t* F;        // [B, K+1] or null
+  const float* alpha;      // [B]: plan computed in-kernel when F is null
+  int fanout_mode;
+  int B, K, V, budget, mode, n_slices, chunk, units_per_row;
+  int draws;               // kernel 2 runs (verify always; reweight: draft tokens drawn)
+  float T, C;
+  // verify outputs
+  int32_t* n_accepted;
+  int32_t* bonus;
+  int32_t* out_tokens;
+  float* accept_prob;
+  float* residual_mass;
+  int32_t* status;
+  int32_t* c_offsets;
+  int32_t* c_tokens;
+  const int32_t* c_payload;
+  uint8_t* c_hit;
+  int32_t* c_slot;
+  int32_t* c_next;
+  unsigned long long fallback_seed;
+  // reweight outputs
+  int32_t* topf_tokens;
+  int32_t* offsets;
+  float* Z;
+  float* q_lse;
+  int32_t* draft_tokens;
+  // workspace
+  SlicePart* parts;
+  UnitState* ustate;
+  DrawPart* dparts;
+  RowState* rstate;
+  int32_t* arrive1;
+  int32_t* row_arrive;
+  int32_t* draw_arrive;
+  int32_t* row_arrive2;
+  int32_t* error;
+};
+
+template <typename TIn>
+struct Elem;
+template <>
+struct Elem<uint16_t> {
+  static constexpr int VE = 8;  // elements per 16-byte vector
+  __device__ static __forceinline__ float at(const uint16_t* p, int i) {
+    return __uint_as_float(static_cast<uint32_t>(p[i]) << 16);
+  }
+  __device__ static __forceinline__ void unpack(const uint4& w, float (&x)[8]) {
+    x[0] = bf16_lo(w.x); x[1] = bf16_hi(w.x); x[2] = bf16_lo(w.y); x[3] = bf16_hi(w.y);
+    x[4] = bf16_lo(w.z); x[5] = bf16_hi(w.z); x[6] = bf16_lo(w.w); x[7] = bf16_hi(w.w);
+  }
+  __device__ static __forceinline__ uint16_t neg_inf() { return 0xFF80u; }
+};
+
+// Streaming loads of one 16-byte vector (read-only path).
+__device__ __forceinline__ uint4 ld_vec(const void* p) { return __ldg(reinterpret_cast<const uint4*>(p)); }
+template <>
+struct Elem<float> {
+  static constexpr int VE = 4;
+  __device__ static __forceinline__ float at(const float* p, int i) { return p[i]; }
+  __device__ static __forceinline__ void unpack(const uint4& w, float (&x)[4]) {
+    x[0] = __uint_as_float(w.x); x[1] = __uint_as_float(w.y);
+    x[2] = __uint_as_float(w.z); x[3] = __uint_as_float(w.w);
+  }
+  __device__ static __forceinline__ float neg_inf() { return -__int_as_float(0x7F800000); }
+};
+
+// Vocab elements [v0, v0 + VE) of the row that starts at element `rb` of
+// `base`; elements at or beyond v_end read as -inf.  Aligned: one 16-byte
+// load (rb, v0 multiples of VE and v0 + VE <= v_end).
+template <typename TIn, bool kAligned>
+__device__ __forceinline__ void load_group(const TIn* __restrict__ base, long long rb, int v0, int v_end,
+                                           float (&x)[Elem<TIn>::VE]) {
+  constexpr int VE = Elem<TIn>::VE;
+  if constexpr (kAligned) {
+    Elem<TIn>::unpack(ld_vec(base + rb + v0), x);
+  } else {
+#pragma unroll
+    for (int i = 0; i < VE; ++i)
+      x[i] = (v0 + i < v_end) ? Elem<TIn>::at(base + rb, v0 + i) : -INFINITY;
+  }
+}
+
+// One vector of logits into a thread's running state.  Softmax: the running
+// maximum m, the sum s of exp2((x - m) c) rescaled when m grows, and
+// nmc = -m c.  Greedy: the running maximum and the lowest id holding it.
+template <bool kGreedy>
+__device__ __forceinline__ float consume_bf16(const uint4 w, int vbase, float c, float& m, float& s, float& nmc,
+                                              int& arg, int& nan_seen) {
+  const uint32_t m2 = bf16x2_max_nan(bf16x2_max_nan(w.x, w.y), bf16x2_max_nan(w.z, w.w));
+  const float vmax = fmax_nan(bf16_lo(m2), bf16_hi(m2));
+  if constexpr (kGreedy) {
+    nan_seen |= vmax != vmax;
+    if (vmax > m) {
+      m = vmax;
+      float x[8];
+      Elem<uint16_t>::unpack(w, x);
+#pragma unroll
+      for (int i = 7; i >= 0; --i)
+        if (x[i] == vmax) arg = vbase + i;
+    }
+  } else {
+    if (!(vmax <= m)) {  // a new maximum (or a NaN, which then sticks)
+      const float nm = fmax_nan(m, vmax);
+      s = (m == -INFINITY) ? 0.f : s * ex2((m - nm) * c);
+      m = nm;
+      nmc = -m * c;
+    }
+    const float e0 = ex2(fmaf(bf16_lo(w.x), c, nmc)) + ex2(fmaf(bf16_hi(w.x), c, nmc));
+    const float e1 = ex2(fmaf(bf16_lo(w.y), c, nmc)) + ex2(fmaf(bf16_hi(w.y), c, nmc));
+    const float e2 = ex2(fmaf(bf16_lo(w.z), c, nmc)) + ex2(fmaf(bf16_hi(w.z), c, nmc));
+    const float e3 = ex2(fmaf(bf16_lo(w.w), c, nmc)) + ex2(fmaf(bf16_hi(w.w), c, nmc));
+    s += (e0 + e1) + (e2 + e3);
+  }
+  return vmax;
+}
+
+template <int VE, bool kGreedy>
+__device__ __forceinline__ float consume_f(const float (&x)[VE], int vbase, float c, float& m, float& s, float& nmc,
+                                           int& arg, int& nan_seen) {
+  float vmax = x[0];
+#pragma unroll
+  for (int i = 1; i < VE; ++i) vmax = fmax_nan(vmax, x[i]);
+  if constexpr (kGreedy) {
+    nan_seen |= vmax != vmax;
+    if (vmax > m) {
+      m = vmax;
+#pragma unroll
+      for (int i = VE - 1; i >= 0; --i)
+        if (x[i] == vmax) arg = vbase + i;
+    }
+  } else {
+    if (!(vmax <= m)) {
+      const float nm = fmax_nan(m, vmax);
+      s = (m == -INFINITY) ? 0.f : s * ex2((m - nm) * c);
+      m = nm;
+      nmc = -m * c;
+    }
+    float acc = 0.f;
+#pragma unroll
+    for (int i = 0; i < VE; ++i) acc += ex2(fmaf(x[i], c, nmc));
+    s += acc;
+  }
+  return vmax;
+}
+
+// Greedy merge: the larger maximum, ties to the lower id (commutative).
+__device__ __forceinline__ void merge_arg(float& m, int& arg, float m2, int arg2) {
+  if (m2 > m || (m2 == m && arg2 < arg)) { m = m2; arg = arg2; }
+  else if (m2 != m2) { m = m2; }
+}
+
+// Merge two (max, sum) pairs taken relative to their own maxima.
+__device__ __forceinline__ void merge_ms(float& m, float& s, float m2, float s2, float c) {
+  const float M = fmax_nan(m, m2);
+  const float a = (m == -INFINITY) ? 0.f : s * ex2((m - M) * c);
+  const float b = (m2 == -INFINITY) ? 0.f : s2 * ex2((m2 - M) * c);
+  m = M;
+  s = a + b;
+}
+
+// Exact top-F of a whole row, read from global memory by one CTA: a radix
+// select on the 32-bit order key (four 8-bit digits), ties at the threshold
+// taken in token-id order, then the F winners ranked by (key, id) in place.
+// Used when the shared-memory candidate filter cannot bound the set (many
+// ties, F large).  `hist` needs 256 ints; the result is sel[0 .. F).
+template <typename TIn>
+__device__ void topf_exact_global(const TIn* row, int V, int F, Cand* sel, int32_t* hist, int tid) {
+  __shared__ uint32_t s_prefix, s_mask;
+  __shared__ int32_t s_remaining, s_napp, s_tie_base[kThreads + 1];
+  if (tid == 0) { s_prefix = 0u; s_mask = 0u; s_remaining = F; s_napp = 0; }
+  __syncthreads();
+  for (int level = 0; level < 4; ++level) {
+    const int shift = 24 - 8 * level;
+    for (int i = tid; i < 256; i += kThreads) hist[i] = 0;
+    __syncthreads();
+    const uint32_t prefix = s_prefix, mask = s_mask;
+    for (int v = tid; v < V; v += kThreads) {
+      const uint32_t k = ord_key(Elem<TIn>::at(row, v));
+      if ((k & mask) == prefix) atomicAdd(&hist[(k >> shift) & 255u], 1);
+    }
+    __syncthreads();
+    if (tid == 0) {
+      int cum = 0, rem = s_remaining, d = 255;
+      for (; d > 0; --d) {
+        if (cum + hist[d] >= rem) break;
+        cum += hist[d];
+      }
+      s_remaining = rem - cum;
+      s_prefix = prefix | (static_cast<uint32_t>(d) << shift);
+      s_mask = mask | (255u << shift);
+    }
+    __syncthreads();
+  }
+  const uint32_t t = s_prefix;
+  const int need_eq = s_remaining;
+  // Ties in token order: each thread owns a contiguous chunk of the row.
+  const int per = (V + kThreads - 1) / kThreads;
+  const int lo = min(V, tid * per), hi = min(V, lo + per);
+  int my_eq = 0;
+  for (int v = lo; v < hi; ++v) my_eq += (ord_key(Elem<TIn>::at(row, v)) == t);
+  s_tie_base[tid + 1] = my_eq;
+  __syncthreads();
+  if (tid == 0) {
+    s_tie_base[0] = 0;
+    for (int i = 1; i <= kThreads; ++i) s_tie_base[i] += s_tie_base[i - 1];
+  }
+  __syncthreads();
+  int tie_rank = s_tie_base[tid];
+  for (int v = lo; v < hi; ++v) {
+    const float x = Elem<TIn>::at(row, v);
+    const uint32_t k = ord_key(x);
+    if (k > t) {
+      const int pos = atomicAdd(&s_napp, 1);
+      if (pos < F) sel[pos] = Cand{x, v};
+    } else if (k == t) {
+      if (tie_rank < need_eq) {
+        const int pos = atomicAdd(&s_napp, 1);
+        if (pos < F) sel[pos] = Cand{x, v};
+      }
+      ++tie_rank;
+    }
+  }
+  __syncthreads();
+  // Rank in place: every thread keeps its (at most two) winners in registers.
+  constexpr int kPer = kSelCap / kThreads;
+  Cand mine[kPer];
+  int rk[kPer];
+#pragma unroll
+  for (int q = 0; q < kPer; ++q) {
+    const int i = tid + q * kThreads;
+    rk[q] = -1;
+    if (i < F) {
+      mine[q] = sel[i];
+      const unsigned long long key = rank_key(mine[q].x, mine[q].idx);
+      int r = 0;
+      for (int k2 = 0; k2 < F; ++k2) r += rank_key(sel[k2].x, sel[k2].idx) > key;
+      rk[q] = r;
+    }
+  }
+  __syncthreads();
+#pragma unroll
+  for (int q = 0; q < kPer; ++q)
+    if (rk[q] >= 0) sel[rk[q]] = mine[q];
+  __syncthreads();
+}
+
+// Fan-out plan of one row ([ZH] section 2 challenge 1; [NL] section 3A):
+// P(k) = alpha^k (1 - alpha) for k < K, P(K) = alpha^K, quotas budget * P(k)
+// rounded by largest remainder (ties to the smaller k); uniform control:
+// floor(budget / (K+1)) each, remainder to the smallest k.  fp64 with every
+// product and difference rounded on its own (no fused multiply-add), so the
+// result is the same integer plan on every device and host.  alpha outside
+// [0, 1] yields F[0] = -1 (a plan the verify rejects).
+__device__ __forceinline__ void fanout_row(float alpha_f, int K, int budget, int mode, int32_t* f) {
+  if (mode == SSD_FANOUT_UNIFORM) {
+    for (int k = 0; k <= K; ++k) f[k] = budget / (K + 1) + (k < budget % (K + 1) ? 1 : 0);
+    return;
+  }
+  const double al = static_cast<double>(alpha_f);
+  if (!(al >= 0.0 && al <= 1.0)) {
+    f[0] = -1;
+    for (int k = 1; k <= K; ++k) f[k] = 0;
+    return;
+  }
+  double frac[SSD_MAX_K + 1];
+  bool taken[SSD_MAX_K + 1];
+  double run = 1.0;
+  long long assigned = 0;
+  for (int k = 0; k <= K; ++k) {
+    double P;
+    if (k < K) {
+      P = __dmul_rn(run, __dsub_rn(1.0, al));
+      run = __dmul_rn(run, al);
+    } else {
+      P = run;
+    }
+    const double quota = __dmul_rn(static_cast<double>(budget), P);
+    const double fl = floor(quota);
+    f[k] = static_cast<int32_t>(fl);
+    frac[k] = __dsub_rn(quota, fl);
+    taken[k] = false;
+    assigned += f[k];
+  }
+  long long rem = budget - assigned;
+  while (rem > 0) {
+    int best = -1;
+    for (int k = 0; k <= K; ++k)
+      if (!taken[k] && (best < 0 || frac[k] > frac[best])) best = k;
+    if (best < 0) {
+      for (int k = 0; k <= K; ++k) taken[k] = false;
+      continue;
+    }
+    taken[best] = true;
+    f[best] += 1;
+    --rem;
+  }
+}
+
+
+// Ring of bulk copies that streams one slice of up to two rows of a unit
+// through shared memory, chunk by chunk (one 16-byte vector per thread per row
+// and chunk).  Thread 0 issues and polls; the other threads sleep in the CTA
+// barrier and then take one acquiring look at the stage's phase.
+template <typename TIn>
+struct Ring {
+  unsigned char* buf;
+  uint64_t* full;
+  const TIn* row0;
+  const TIn* row1;
+  int nrows, e0, nvec, nch, n_issued;
+
+  __device__ __forceinline__ unsigned char* stage(int slot, int r) const {
+    return buf + (static_cast<size_t>(slot) * 2 + r) * (kChunkVecs * 16);
+  }
+  __device__ __forceinline__ void issue(int c) {
+    constexpr int VE = 16 / sizeof(TIn);
+    const int slot = c % kStages;
+    const int v0 = c * kChunkVecs;
+    const int nv = min(kChunkVecs, nvec - v0);
+    mbar_arrive_expect_tx(&full[slot], static_cast<uint32_t>(nv) * 16u * static_cast<uint32_t>(nrows));
+    bulk_copy_g2s(stage(slot, 0), row0 + e0 + v0 * VE, static_cast<uint32_t>(nv) * 16u, &full[slot]);
+    if (nrows > 1) bulk_copy_g2s(stage(slot, 1), row1 + e0 + v0 * VE, static_cast<uint32_t>(nv) * 16u, &full[slot]);
+    n_issued = c + 1;
+  }
+  __device__ __forceinline__ void start(int tid) {
+    n_issued = 0;
+    if (tid == 0) {
+      for (int s = 0; s < kStages; ++s) mbar_init(&full[s], 1);
+      mbar_init_fence();
+    }
+    __syncthreads();
+    if (tid == 0)
+      for (int c = 0; c < min(kStages, nch); ++c) issue(c);
+  }
+  // Chunk c is ready for every thread; the barrier also marks chunk c - 1
+  // consumed, so its stage is refilled.
+  __device__ __forceinline__ void acquire(int c, int tid, int& tmo) {
+    if (tid == 0 && !mbar_wait_bounded(&full[c % kStages], (c / kStages) & 1, kMaxPolls)) tmo = 1;
+    __syncthreads();
+    if (tid == 0 && c > 0 && c - 1 + kStages < nch) issue(c - 1 + kStages);
+    if (tid != 0 && !mbar_try_wait(&full[c % kStages], (c / kStages) & 1, 0u)) tmo = 1;
+  }
+  __device__ __forceinline__ uint4 vec(int c, int r, int tid) const {
+    return *reinterpret_cast<const uint4*>(stage(c % kStages, r) + tid * 16);
+  }
+  // Never leave a copy in flight (only a timed-out wait can leave one).
+  __device__ __forceinline__ void drain(int tid, int tmo) {
+    if (tmo && tid == 0)
+      for (int c = max(0, n_issued - kStages); c < n_issued; ++c)
+        mbar_wait_bounded(&full[c % kStages], (c / kStages) & 1, kMaxPolls);
+  }
+};
+
+// Roles of a unit: its p row (verify), its q row (draft, draft_next or guess).
+template <typename TIn>
+__device__ __forceinline__ void unit_rows(const Args& a, int b, int j, const TIn*& baseP, long long& rbP,
+                                          const TIn*& baseQ, long long& rbQ) {
+  const int K = a.K, V = a.V;
+  baseP = nullptr;
+  baseQ = nullptr;
+  rbP = rbQ = 0;
+  if (a.mode == kModeVerify) {
+    baseP = static_cast<const TIn*>(a.target);
+    rbP = (static_cast<long long>(b) * (K + 1) + j) * V;
+    if (j < K) {
+      baseQ = static_cast<const TIn*>(a.draft);
+      rbQ = (static_cast<long long>(b) * K + j) * V;
+    } else if (a.draft_next) {
+      baseQ = static_cast<const TIn*>(a.draft_next);
+      rbQ = static_cast<long long>(b) * V;
+    }
+  } else {
+    if (j < K) {
+      baseQ = static_cast<const TIn*>(a.draft);
+      rbQ = (static_cast<long long>(b) * K + j) * V;
+    } else {
+      baseQ = static_cast<const TIn*>(a.guess);
+      rbQ = static_cast<long long>(b) * a.guess_stride;
+    }
+  }
+}
+
+// The row's fan-out plan into shared memory (thread 0): F when given, else
+// planned from alpha.  Returns nothing; callers check Σ F = budget, 0 <= F <= V.
+__device__ __forceinline__ void load_plan(const Args& a, int b, int32_t* s_F) {
+  if (a.F) {
+    for (int k = 0; k <= a.K; ++k) s_F[k] = __ldg(a.F + static_cast<long long>(b) * (a.K + 1) + k);
+  } else {
+    fanout_row(__ldg(a.alpha + b), a.K, a.budget, a.fanout_mode, s_F);
+  }
+}
+
+// Shared memory of kernel 1.
+struct Smem1 {
+  uint64_t full[kStages];
+  float wred[kWarps][4];
+  int32_t wint[kWarps][2];
+  float gmax[kMaxGroups];
+  int32_t hist[256];
+  int32_t s_F[SSD_MAX_K + 1];
+  float tau, MP, SP, MQ, SQ, QS, bx;
+  int32_t bi, argP, argQ, n_total, slow, tmo, n_raw, is_last, is_last_row, pad;
+  int32_t cand_off[kMaxSlices + 1];
+  Cand raw[kCandCap];
+  Cand buf[kGatherCap + kSelCap];  // the unit's gathered candidates, then its sorted top-F
+};
+
+template <typename TIn, bool kAligned, bool kGreedy>
+__global__ void __launch_bounds__(kThreads, kMinBlocks) ssd_stats_kernel(const __grid_constant__ Args a) {
+  constexpr int VE = Elem<TIn>::VE;
+  extern __shared__ __align__(128) unsigned char ring_buf[];
+  __shared__ __align__(16) Smem1 sm;
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int S = a.n_slices;
+  const int order = blockIdx.x / S, slice = blockIdx.x % S;
+  const int upr = a.units_per_row;
+  const int b = order % a.B, j = (upr - 1) - order / a.B;  // decreasing position order
+  const int K = a.K, V = a.V;
+  const bool verify = a.mode == kModeVerify;
+  const long long u = static_cast<long long>(b) * (K + 1) + j;
+
+  const TIn *baseP, *baseQ;
+  long long rbP, rbQ;
+  unit_rows<TIn>(a, b, j, baseP, rbP, baseQ, rbQ);
+  const bool hasP = baseP != nullptr, hasQ = baseQ != nullptr;
+  const bool srcQ = hasQ;  // the top-F source row: q_j, else p_j
+  const bool has_d = verify && j < K;
+
+  // ---- slice [e0, e1) of the rows, vectors of VE elements --------------------------
+  const int e0 = slice * a.chunk;
+  const int e1 = min(V, e0 + a.chunk);
+  const int n = max(0, e1 - e0);
+  const int nvec = (n + VE - 1) / VE;
+  const int nch = (nvec + kChunkVecs - 1) / kChunkVecs;
+  Ring<TIn> ring;
+  ring.buf = ring_buf;
+  ring.full = sm.full;
+  ring.row0 = hasP ? baseP + rbP : baseQ + rbQ;
+  ring.row1 = baseQ + rbQ;
+  ring.nrows = (hasP ? 1 : 0) + (hasQ ? 1 : 0);
+  ring.e0 = e0;
+  ring.nvec = nvec;
+  ring.nch = nch;
+  const int slotP = 0, slotQ = hasP ? 1 : 0;
+  if constexpr (kAligned) ring.start(tid);
+
+  const bool has_plan = a.F != nullptr || a.alpha != nullptr;
+  if (tid == 0 && has_plan) load_plan(a, b, sm.s_F);
+  int flags = 0, d = -1;
+  float u_self = 0.f;
+  if (has_d) {
+    d = __ldg(a.tokens + static_cast<long long>(b) * K + j);
+    if (d < 0 || d >= V) flags |= SSD_ROW_BAD_TOKEN;
+  }
+  if (verify) {
+    u_self = __ldg(a.uniforms + static_cast<long long>(b) * (K + 1) + j);
+    if (!(u_self >= 0.f && u_self < 1.f)) flags |= SSD_ROW_BAD_UNIFORM;
+  } else if (j < K && a.uniforms) {
+    const float ud = __ldg(a.uniforms + static_cast<long long>(b) * K + j);
+    if (!(ud >= 0.f && ud < 1.f)) flags |= SSD_ROW_BAD_UNIFORM;
+  }
+  __syncthreads();
+  int Fj = 0, seg_off = 0, plan_bad = 0;
+  if (has_plan) {
+    long long sum = 0;
+    for (int k = 0; k <= K; ++k) {
+      const int f = sm.s_F[k];
+      if (f < 0 || f > V) plan_bad = 1;
+      if (k < j) seg_off += f;
+      sum += f;
+    }
+    if (sum != a.budget) plan_bad = 1;
+    Fj = plan_bad ? 0 : sm.s_F[j];
+  }
+  if (plan_bad) flags |= SSD_ROW_BAD_PLAN;
+  const bool want_topf = has_plan && Fj > 0;
+  const float cT = kGreedy ? 0.f : kLog2e / a.T;
+
+  // ---- the stream: online max / exp-sum (or greedy argmax) of both rows ----------
+  float mP = -INFINITY, sP = 0.f, nmP1 = 0.f, mQ = -INFINITY, sQ = 0.f, nmQ1 = 0.f;
+  int argP = INT_MAX, argQ = INT_MAX, nan_seen = 0, tmo = 0;
+  float vm1 = -INFINITY, vm2 = -INFINITY;  // top two vector maxima of the source row
+  int g1 = -1;
+  uint4 keep = make_uint4(0u, 0u, 0u, 0u);  // the source vector holding vm1
+  for (int c = 0; c < nch; ++c) {
+    if constexpr (kAligned) ring.acquire(c, tid, tmo);
+    const int g = c * kChunkVecs + tid;
+    if (g < nvec) {
+      const int vbase = e0 + g * VE;
+      float vsrc;
+      uint4 wsrc = make_uint4(0u, 0u, 0u, 0u);
+      if constexpr (kAligned && sizeof(TIn) == 2) {
+        float vp = -INFINITY;
+        uint4 wq = make_uint4(0u, 0u, 0u, 0u), wp = wq;
+        if (hasP) { wp = ring.vec(c, slotP, tid); vp = consume_bf16<kGreedy>(wp, vbase, cT, mP, sP, nmP1, argP, nan_seen); }
+        float vq = -INFINITY;
+        if (hasQ) { wq = ring.vec(c, slotQ, tid); vq = consume_bf16<kGreedy>(wq, vbase, cT, mQ, sQ, nmQ1, argQ, nan_seen); }
+        vsrc = srcQ ? vq : vp;
+        wsrc = srcQ ? wq : wp;
+      } else {
+        float x[VE];
+        float vp = -INFINITY, vq = -INFINITY;
+        uint4 wp = make_uint4(0u, 0u, 0u, 0u), wq = wp;
+        if (hasP) {
+          if constexpr (kAligned) { wp = ring.vec(c, slotP, tid); Elem<TIn>::unpack(wp, x); }
+          else load_group<TIn, false>(baseP, rbP, vbase, e1, x);
+          vp = consume_f<VE, kGreedy>(x, vbase, cT, mP, sP, nmP1, argP, nan_seen);
+        }
+        if (hasQ) {
+          if constexpr (kAligned) { wq = ring.vec(c, slotQ, tid); Elem<TIn>::unpack(wq, x); }
+          else load_group<TIn, false>(baseQ, rbQ, vbase, e1, x);
+          vq = consume_f<VE, kGreedy>(x, vbase, cT, mQ, sQ, nmQ1, argQ, nan_seen);
+        }
+        vsrc = srcQ ? vq : vp;
+        wsrc = srcQ ? wq : wp;
+      }
+      if (vsrc > vm2) {
+        if (vsrc > vm1) { vm2 = vm1; vm1 = vsrc; g1 = g; keep = wsrc; }
+        else vm2 = vsrc;
+      }
+    }
+  }
+  if constexpr (kGreedy) {
+    if (nan_seen) { mP = __int_as_float(0x7FC00000); mQ = mP; }
+  }
+  sm.gmax[tid] = vm1;
+  if (tid == 0) sm.n_raw = 0;
+
+  // ---- slice reduction: butterfly within each warp, then over the warps ----------
+  if constexpr (kGreedy) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      merge_arg(mP, argP, __shfl_xor_sync(0xFFFFFFFFu, mP, o), __shfl_xor_sync(0xFFFFFFFFu, argP, o));
+      merge_arg(mQ, argQ, __shfl_xor_sync(0xFFFFFFFFu, mQ, o), __shfl_xor_sync(0xFFFFFFFFu, argQ, o));
+    }
+    if (lane == 0) {
+      sm.wred[warp][0] = mP; sm.wred[warp][2] = mQ;
+      sm.wint[warp][0] = argP; sm.wint[warp][1] = argQ;
+    }
+  } else {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      merge_ms(mP, sP, __shfl_xor_sync(0xFFFFFFFFu, mP, o), __shfl_xor_sync(0xFFFFFFFFu, sP, o), cT);
+      merge_ms(mQ, sQ, __shfl_xor_sync(0xFFFFFFFFu, mQ, o), __shfl_xor_sync(0xFFFFFFFFu, sQ, o), cT);
+    }
+    if (lane == 0) {
+      sm.wred[warp][0] = mP; sm.wred[warp][1] = sP;
+      sm.wred[warp][2] = mQ; sm.wred[warp][3] = sQ;
+    }
+  }
+  const bool fast_ok = want_topf && Fj <= kMaxGroups;
+  tmo = __syncthreads_or(tmo);
+  SlicePart* part = a.parts + u * S + slice;
+  if (warp == 0) {
+    float m1 = -INFINITY, s1 = 0.f, m2 = -INFINITY, s2 = 0.f;
+    int a1 = INT_MAX, a2 = INT_MAX;
+    if (lane < kWarps) {
+      m1 = sm.wred[lane][0]; s1 = sm.wred[lane][1]; m2 = sm.wred[lane][2]; s2 = sm.wred[lane][3];
+      if constexpr (kGreedy) { a1 = sm.wint[lane][0]; a2 = sm.wint[lane][1]; }
+    }
+#pragma unroll
+    for (int o = kWarps / 2; o > 0; o >>= 1) {
+      if constexpr (kGreedy) {
+        merge_arg(m1, a1, __shfl_xor_sync(0xFFFFFFFFu, m1, o), __shfl_xor_sync(0xFFFFFFFFu, a1, o));
+        merge_arg(m2, a2, __shfl_xor_sync(0xFFFFFFFFu, m2, o), __shfl_xor_sync(0xFFFFFFFFu, a2, o));
+      } else {
+        merge_ms(m1, s1, __shfl_xor_sync(0xFFFFFFFFu, m1, o), __shfl_xor_sync(0xFFFFFFFFu, s1, o), cT);
+        merge_ms(m2, s2, __shfl_xor_sync(0xFFFFFFFFu, m2, o), __shfl_xor_sync(0xFFFFFFFFu, s2, o), cT);
+      }
+    }
+    if (lane == 0) {
+      part->mP = m1; part->sP = kGreedy ? 0.f : s1;
+      part->mQ = m2; part->sQ = kGreedy ? 0.f : s2;
+      part->argP = a1; part->argQ = a2;
+      part->timeout = tmo;
+    }
+  } else if (warp == 1) {
+    // This slice's threshold: the F-th largest of its thread maxima bounds the
+    // slice's own top-F (hence its share of the unit's top-F) from below.
+    float t = -INFINITY;
+    if (fast_ok) {
+      uint32_t keys[kMaxGroups / 32];
+#pragma unroll
+      for (int i = 0; i < kMaxGroups / 32; ++i) keys[i] = ord_key(sm.gmax[lane + 32 * i]);
+      t = key_to_float(warp_kth_largest(keys, Fj, sizeof(TIn) == 2 ? 16 : 32));
+    }
+    if (lane == 0) sm.tau = t;
+  }
+  __syncthreads();
+  const float tau = sm.tau;
+
+  // Local candidates: the elements at or above tau.  A thread whose second
+  // vector maximum is below tau holds them all in its kept vector.
+  if (fast_ok && vm1 >= tau && vm1 == vm1) {
+    if (kAligned && vm2 < tau) {
+      float x[VE];
+      Elem<TIn>::unpack(keep, x);
+#pragma unroll
+      for (int i = 0; i < VE; ++i) {
+        const int v = e0 + g1 * VE + i;
+        if (x[i] >= tau && v < e1) {
+          const int pos = atomicAdd(&sm.n_raw, 1);
+          if (pos < kCandCap) sm.raw[pos] = Cand{x[i], v};
+        }
+      }
+    } else {
+      const TIn* bs = srcQ ? baseQ : baseP;
+      const long long rs = srcQ ? rbQ : rbP;
+      for (int c = 0; c < nch; ++c) {
+        const int g = c * kChunkVecs + tid;
+        if (g < nvec) {
+          float x[VE];
+          load_group<TIn, kAligned>(bs, rs, e0 + g * VE, e1, x);
+#pragma unroll
+          for (int i = 0; i < VE; ++i) {
+            const int v = e0 + g * VE + i;
+            if (x[i] >= tau && v < e1) {
+              const int pos = atomicAdd(&sm.n_raw, 1);
+              if (pos < kCandCap) sm.raw[pos] = Cand{x[i], v};
+            }
+          }
+        }
+      }
+    }
+  }
+  __syncthreads();
+  {
+    // Sort the local candidates; publish the first min(count, F) of them.
+    const int nr = min(sm.n_raw, kCandCap);
+    const int keepn = min(min(nr, Fj), kCandSlice);
+    for (int i = tid; i < nr; i += kThreads) {
+      const Cand ci = sm.raw[i];
+      const unsigned long long key = rank_key(ci.x, ci.idx);
+      int r = 0;
+      for (int k2 = 0; k2 < nr; ++k2) r += rank_key(sm.raw[k2].x, sm.raw[k2].idx) > key;
+      if (r < keepn) part->cand[r] = ci;
+    }
+    if (tid == 0) part->n_cand = sm.n_raw;
+  }
+  __threadfence();
+  __syncthreads();
+  if constexpr (kAligned) ring.drain(tid, tmo);
+  if (tid == 0) sm.is_last = atomicAdd(a.arrive1 + u, 1) == S - 1;
+  __syncthreads();
+  if (!sm.is_last) return;
+  __threadfence();
+
+  // =============== the unit's finalizer: the last slice to arrive ===================
+  const SlicePart* parts = a.parts + u * S;
+  if (warp == 0) {
+    // Butterfly over the slices (lanes >= S hold neutral values): bit-identical
+    // results whichever CTA finalizes.
+    float mp = -INFINITY, sp = 0.f, mq = -INFINITY, sq = 0.f;
+    int ap = INT_MAX, aq = INT_MAX, nc = 0, to = 0;
+    if (lane < S) {
+      mp = __ldcg(&parts[lane].mP); sp = __ldcg(&parts[lane].sP);
+      mq = __ldcg(&parts[lane].mQ); sq = __ldcg(&parts[lane].sQ);
+      ap = __ldcg(&parts[lane].argP); aq = __ldcg(&parts[lane].argQ);
+      nc = __ldcg(&parts[lane].n_cand); to = __ldcg(&parts[lane].timeout);
+    }
+    const int cnt = min(min(nc, Fj), kCandSlice);
+#pragma unroll
+    for (int o = kMaxSlices / 2; o > 0; o >>= 1) {
+      if constexpr (kGreedy) {
+        merge_arg(mp, ap, __shfl_xor_sync(0xFFFFFFFFu, mp, o), __shfl_xor_sync(0xFFFFFFFFu, ap, o));
+        merge_arg(mq, aq, __shfl_xor_sync(0xFFFFFFFFu, mq, o), __shfl_xor_sync(0xFFFFFFFFu, aq, o));
+      } else {
+        merge_ms(mp, sp, __shfl_xor_sync(0xFFFFFFFFu, mp, o), __shfl_xor_sync(0xFFFFFFFFu, sp, o), cT);
+        merge_ms(mq, sq, __shfl_xor_sync(0xFFFFFFFFu, mq, o), __shfl_xor_sync(0xFFFFFFFFu, sq, o), cT);
+      }
+    }
+    int incl = cnt;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    const int total = __shfl_sync(0xFFFFFFFFu, incl, 31);
+    const unsigned over = __ballot_sync(0xFFFFFFFFu, nc > kCandCap || (nc > kCandSlice && Fj > kCandSlice));
+    const unsigned anyto = __ballot_sync(0xFFFFFFFFu, to != 0);
+    if (lane < S) sm.cand_off[lane] = incl - cnt;
+    if (lane == 0) {
+      sm.MP = mp; sm.SP = sp; sm.MQ = mq; sm.SQ = sq; sm.argP = ap; sm.argQ = aq;
+      sm.cand_off[S] = total;
+      sm.n_total = total;
+      sm.tmo = anyto ? 1 : 0;
+      sm.slow = over || total > kGatherCap || total < Fj;
+    }
+  }
+  __syncthreads();
+  const float MP = sm.MP, MQ = sm.MQ, SP = sm.SP, SQ = sm.SQ;
+  if (sm.tmo) flags |= kFlagTimeout;
+  if (hasP && !(MP > -INFINITY && MP < INFINITY)) flags |= SSD_ROW_NONFINITE;
+  if (hasQ && !(MQ > -INFINITY && MQ < INFINITY)) flags |= SSD_ROW_NONFINITE;
+  const bool valid = (flags & SSD_ROW_INVALID) == 0;
+  const bool slow = want_topf && valid && (!fast_ok || sm.slow != 0);
+  Cand* sel = sm.buf + kGatherCap;
+  const float nmP = -MP * cT, nmQ = -MQ * cT;
+
+  // ---- exact top-F: global ranks by binary search in the sorted slice lists --------
+  if (want_topf && valid && !slow) {
+    const int N = sm.n_total;
+    for (int i = tid; i < N; i += kThreads) {
+      int c = 0;
+      while (c + 1 < S && sm.cand_off[c + 1] <= i) ++c;
+      const Cand* src = &parts[c].cand[i - sm.cand_off[c]];
+      sm.buf[i] = Cand{__ldcg(&src->x), __ldcg(&src->idx)};
+    }
+    __syncthreads();
+    for (int i = tid; i < N; i += kThreads) {
+      int c = 0;
+      while (c + 1 < S && sm.cand_off[c + 1] <= i) ++c;
+      const Cand ci = sm.buf[i];
+      const unsigned long long key = rank_key(ci.x, ci.idx);
+      int r = i - sm.cand_off[c];  // entries ahead of it in its own list
+      for (int c2 = 0; c2 < S; ++c2) {
+        if (c2 == c) continue;
+        int lo = sm.cand_off[c2], hi = sm.cand_off[c2 + 1];  // count keys > key (descending list)
+        while (lo < hi) {
+          const int mid = (lo + hi) >> 1;
+          if (rank_key(sm.buf[mid].x, sm.buf[mid].idx) > key) lo = mid + 1;
+          else hi = mid;
+        }
+        r += lo - sm.cand_off[c2];
+      }
+      if (r < Fj) sel[r] = ci;
+    }
+  }
+  if (slow) {
+    const TIn* row = srcQ ? baseQ + rbQ : baseP + rbP;
+    topf_exact_global<TIn>(row, V, Fj, sel, sm.hist, tid);
+  }
+  __syncthreads();
+
+  // Q_S in a fixed order, and the top-F boundary.
+  if (warp == 0) {
+    float qs = 0.f;
+    if (want_topf && valid) {
+      if constexpr (!kGreedy) {
+        for (int i = lane; i < Fj; i += 32) qs += ex2(fmaf(sel[i].x, cT, srcQ ? nmQ : nmP));
+      }
+    }
+    qs = warp_sum(qs);
+    if (lane == 0) {
+      sm.QS = qs;
+      sm.bx = (want_topf && valid) ? sel[Fj - 1].x : INFINITY;
+      sm.bi = (want_topf && valid) ? sel[Fj - 1].idx : -1;
+    }
+  }
+  __syncthreads();
+
+  // ---- Saguaro normaliser and the accept test --------------------------------------
+  const float C = a.C;
+  float Z = 1.f;
+  if (!kGreedy && want_topf && valid) Z = 1.f - (1.f - C) * (sm.QS / (srcQ ? SQ : SP));
+  const float bx = sm.bx;
+  const int bi = sm.bi;
+  float acc = 0.f, amargin = INFINITY;
+  int rejected = 0;
+  if (has_d && valid) {
+    if constexpr (kGreedy) {
+      acc = (d == sm.argP) ? 1.f : 0.f;
+      rejected = d != sm.argP;
+    } else {
+      const float xdP = Elem<TIn>::at(baseP + rbP, d);
+      const float xdQ = Elem<TIn>::at(baseQ + rbQ, d);
+      const float pd = ex2(fmaf(xdP, cT, nmP)) / SP;
+      const float qd = ex2(fmaf(xdQ, cT, nmQ)) / SQ;
+      const bool inS = want_topf && (xdQ > bx || (xdQ == bx && d <= bi));
+      const float qpd = (inS ? C : 1.f) * qd / Z;
+      if (qpd > 0.f) {
+        acc = fminf(1.f, pd / qpd);
+      } else {
+        acc = pd > 0.f ? 1.f : 0.f;
+        flags |= SSD_ROW_ZERO_Q;
+      }
+      rejected = !(u_self < acc);
+      amargin = fabsf(u_self - acc);
+    }
+  }
+
+  // ---- unit outputs ------------------------------------------------------------------
+  int32_t* segdst = nullptr;
+  if (verify) {
+    if (a.c_tokens && !plan_bad) segdst = a.c_tokens + static_cast<long long>(b) * a.budget + seg_off;
+  } else if (!plan_bad) {
+    segdst = a.topf_tokens + static_cast<long long>(b) * a.budget + seg_off;
+  }
+  if (segdst && has_plan)
+    for (int i = tid; i < Fj; i += kThreads) segdst[i] = valid ? sel[i].idx : -1;
+  if (tid == 0) {
+    if (verify && j < K) a.accept_prob[static_cast<long long>(b) * K + j] = valid ? acc : __int_as_float(0x7FC00000);
+    if (!verify && j < K) {
+      const long long o = static_cast<long long>(b) * K + j;
+      const float qlse = kGreedy ? MQ : (MQ * cT + log2f(SQ)) * 0.6931471805599453f;
+      a.Z[o] = valid ? Z : __int_as_float(0x7FC00000);
+      a.q_lse[o] = valid ? qlse : __int_as_float(0x7FC00000);
+      if (a.draft_tokens && (!valid || !a.draws)) a.draft_tokens[o] = valid ? sm.argQ : -1;
+    }
+    UnitState st;
+    st.MP = MP; st.SP = SP; st.MQ = MQ; st.SQ = SQ;
+    st.Z = Z; st.bx = bx; st.a = acc; st.amargin = amargin;
+    st.bi = bi; st.argP = sm.argP; st.argQ = sm.argQ; st.flags = flags;
+    st.rejected = rejected; st.Fj = Fj; st.seg_off = seg_off; st.dmargin = INFINITY;
+    a.ustate[u] = st;
+    a.arrive1[u] = 0;
+  }
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) sm.is_last_row = atomicAdd(a.row_arrive + b, 1) == upr - 1;
+  __syncthreads();
+  if (!sm.is_last_row) return;
+  __threadfence();
+
+  // =============== the row's decision: the last unit of the row to finish ===========
+  if (tid == 0) {
+    const UnitState* us = a.ustate + static_cast<long long>(b) * (K + 1);
+    int fl = 0;
+    for (int k = 0; k < upr; ++k) fl |= __ldcg(&us[k].flags);
+    if (verify) {
+      int kstar = K;
+      float am = INFINITY;
+      for (int k = 0; k < K; ++k) {
+        am = fminf(am, __ldcg(&us[k].amargin));
+        if (__ldcg(&us[k].rejected)) { kstar = k; break; }
+      }
+      RowState rs;
+      rs.kstar = kstar;
+      rs.flags = fl;
+      rs.amargin = am;
+      rs.pad = 0;
+      a.rstate[b] = rs;
+    } else {
+      const bool pbad = (fl & SSD_ROW_BAD_PLAN) != 0;
+      int off = 0;
+      a.offsets[static_cast<long long>(b) * (K + 2)] = 0;
+      for (int k = 0; k <= K; ++k) {
+        off += pbad ? 0 : sm.s_F[k];
+        a.offsets[static_cast<long long>(b) * (K + 2) + k + 1] = off;
+      }
+      if (!a.draws) a.status[b] = fl;
+      else a.rstate[b] = RowState{0, fl, INFINITY, 0};
+    }
+    a.row_arrive[b] = 0;
+  }
+}
+
+// Shared memory of kernel 2.
+struct Smem2 {
+  uint64_t full[kStages];
+  float rs[kMaxChunks][kWarps];
+  float ps[kMaxChunks][kWarps];
+  int32_t s_F[SSD_MAX_K + 1];
+  float tl, total, margin;
+  int32_t cstar, use_p, drawn, is_last, is_last_row, slot, tmo;
+};
+
+// The draw's mass at VE consecutive tokens of vector g of slice [e0, e1).
+template <typename TIn, bool kAligned>
+__device__ __forceinline__ void draw_vals(int draw, const TIn* baseP, long long rbP, const TIn* baseQ, long long rbQ,
+                                          int e0, int e1, int g, const uint4* wp_ring, const uint4* wq_ring,
+                                          float cT, float nmP, float nmQ, float invSP, float wS, float wN, bool check_S,
+                                          float bx, int bi, bool use_p, float (&val)[Elem<TIn>::VE],
+                                          float (&pv)[Elem<TIn>::VE]) {
+  constexpr int VE = Elem<TIn>::VE;
+  float xp[VE], xq[VE];
+  if (draw != kDrawQ) {
+    if (wp_ring) Elem<TIn>::unpack(*wp_ring, xp);
+    else load_group<TIn, kAligned>(baseP, rbP, e0 + g * VE, e1, xp);
+  }
+  if (draw != kDrawP) {
+    if (wq_ring) Elem<TIn>::unpack(*wq_ring, xq);
+    else load_group<TIn, kAligned>(baseQ, rbQ, e0 + g * VE, e1, xq);
+  }
+#pragma unroll
+  for (int i = 0; i < VE; ++i) {
+    float wq = wN;
+    if (check_S) {
+      const int v = e0 + g * VE + i;
+      if (xq[i] > bx || (xq[i] == bx && v <= bi)) wq = wS;
+    }
+    if (draw == kDrawResidual) {
+      const float pp = ex2(fmaf(xp[i], cT, nmP)) * invSP;
+      val[i] = use_p ? pp : fmaxf(pp - ex2(fmaf(xq[i], cT, nmQ)) * wq, 0.f);
+      pv[i] = pp;
+    } else if (draw == kDrawP) {
+      val[i] = ex2(fmaf(xp[i], cT, nmP)) * invSP;
+      pv[i] = 0.f;
+    } else {
+      val[i] = ex2(fmaf(xq[i], cT, nmQ)) * wq;
+      pv[i] = 0.f;
+    }
+  }
+}
+
+template <typename TIn, bool kAligned, bool kGreedy>
+__global__ void __launch_bounds__(kThreads, kMinBlocks) ssd_draw_kernel(const __grid_constant__ Args a) {
+  constexpr int VE = Elem<TIn>::VE;
+  extern __shared__ __align__(128) unsigned char ring_buf[];
+  __shared__ __align__(16) Smem2 sm;
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int S = a.n_slices;
+  const int du = blockIdx.x / S, slice = blockIdx.x % S;
+  const int K = a.K, V = a.V;
+  const bool verify = a.mode == kModeVerify;
+
+  // ---- which unit this row (or draft position) draws from ----------------------------
+  int b, j, rowflags = 0, draw;
+  float amargin = INFINITY;
+  if (verify) {
+    b = du;
+    const RowState rs = a.rstate[b];
+    j = rs.kstar;
+    rowflags = rs.flags;
+    amargin = rs.amargin;
+    draw = j < K ? kDrawResidual : kDrawP;
+  } else {
+    b = du / K;
+    j = du % K;
+    draw = kDrawQ;
+  }
+  const long long u = static_cast<long long>(b) * (K + 1) + j;
+  const UnitState st = a.ustate[u];
+  const bool row_invalid = verify ? (rowflags & SSD_ROW_INVALID) != 0 : (st.flags & SSD_ROW_INVALID) != 0;
+  const bool streams = !kGreedy && !row_invalid;
+  if (!streams && slice != 0) return;
+
+  const TIn *baseP, *baseQ;
+  long long rbP, rbQ;
+  unit_rows<TIn>(a, b, j, baseP, rbP, baseQ, rbQ);
+  if (draw == kDrawP) baseQ = nullptr;  // the full-acceptance draw reads p_K only
+  const int e0 = slice * a.chunk;
+  const int e1 = min(V, e0 + a.chunk);
+  const int n = max(0, e1 - e0);
+  const int nvec = (n + VE - 1) / VE;
+  const int nch = (nvec + kChunkVecs - 1) / kChunkVecs;
+  const bool useP = draw != kDrawQ, useQ = draw != kDrawP;
+  Ring<TIn> ring;
+  ring.buf = ring_buf;
+  ring.full = sm.full;
+  ring.row0 = useP ? baseP + rbP : baseQ + rbQ;
+  ring.row1 = useQ ? baseQ + rbQ : nullptr;
+  ring.nrows = (useP ? 1 : 0) + (useQ ? 1 : 0);
+  ring.e0 = e0;
+  ring.nvec = nvec;
+  ring.nch = nch;
+  const int slotP = 0, slotQ = useP ? 1 : 0;
+  if (kAligned && streams) ring.start(tid);
+
+  const float cT = kGreedy ? 0.f : kLog2e / a.T;
+  const float C = a.C;
+  const float nmP = -st.MP * cT, nmQ = -st.MQ * cT;
+  const float invSP = 1.f / st.SP;
+  const float wS = C / (st.SQ * st.Z), wN = 1.f / (st.SQ * st.Z);
+  const bool check_S = st.Fj > 0 && draw != kDrawP;
+  const float u_draw = verify ? __ldg(a.uniforms + static_cast<long long>(b) * (K + 1) + K)
+                              : __ldg(a.uniforms + static_cast<long long>(b) * K + j);
+  int tmo = 0;
+  DrawPart* dparts = a.dparts + static_cast<long long>(du) * S;
+
+  if (streams) {
+    // ---- this slice's mass per (chunk, warp), in token order ------------------------
+    for (int c = 0; c < nch; ++c) {
+      if constexpr (kAligned) ring.acquire(c, tid, tmo);
+      const int g = c * kChunkVecs + tid;
+      float rsum = 0.f, psum = 0.f;
+      if (g < nvec) {
+        float val[VE], pv[VE];
+        uint4 wp, wq;
+        if constexpr (kAligned) {
+          if (useP) wp = ring.vec(c, slotP, tid);
+          if (useQ) wq = ring.vec(c, slotQ, tid);
+        }
+        draw_vals<TIn, kAligned>(draw, baseP, rbP, baseQ, rbQ, e0, e1, g, kAligned ? &wp : nullptr,
+                                 kAligned ? &wq : nullptr, cT, nmP, nmQ, invSP, wS, wN, check_S, st.bx, st.bi,
+                                 false, val, pv);
+#pragma unroll
+        for (int i = 0; i < VE; ++i) { rsum += val[i]; psum += pv[i]; }
+      }
+      rsum = warp_sum(rsum);
+      psum = warp_sum(psum);
+      if (lane == 0) { sm.rs[c][warp] = rsum; sm.ps[c][warp] = psum; }
+    }
+    tmo = __syncthreads_or(tmo);
+    if (tid == 0) {
+      float R = 0.f, RP = 0.f;
+      for (int c = 0; c < nch; ++c)
+        for (int w = 0; w < kWarps; ++w) { R += sm.rs[c][w]; RP += sm.ps[c][w]; }
+      dparts[slice].R = R;
+      dparts[slice].RP = RP;
+      dparts[slice].timeout = tmo;
+    }
+    for (int i = tid; i < nch * kWarps; i += kThreads) {
+      dparts[slice].rs[i / kWarps][i % kWarps] = sm.rs[i / kWarps][i % kWarps];
+      dparts[slice].ps[i / kWarps][i % kWarps] = sm.ps[i / kWarps][i % kWarps];
+    }
+    __threadfence();
+    __syncthreads();
+    if constexpr (kAligned) ring.drain(tid, tmo);
+    if (tid == 0) sm.is_last = atomicAdd(a.draw_arrive + du, 1) == S - 1;
+    __syncthreads();
+    if (!sm.is_last) return;
+    __threadfence();
+
+    // ============ the draw: the last slice of this unit to arrive ====================
+    if (warp == 0) {
+      float rp = 0.f, pp = 0.f;
+      int to = 0;
+      if (lane < S) {
+        rp = __ldcg(&dparts[lane].R);
+        pp = __ldcg(&dparts[lane].RP);
+        to = __ldcg(&dparts[lane].timeout);
+      }
+      float R = 0.f, RP = 0.f;
+      for (int c = 0; c < S; ++c) {
+        R += __shfl_sync(0xFFFFFFFFu, rp, c);
+        RP += __shfl_sync(0xFFFFFFFFu, pp, c);
+      }
+      const int use_p = (draw == kDrawResidual && !(R > 0.f)) ? 1 : 0;
+      const float total = use_p ? RP : R;
+      const float t = u_draw * total;
+      // crossing slice: the first with prefix + part > t, else the last with mass
+      float run = 0.f, pre = 0.f, prelast = 0.f;
+      int cstar = -1, clast = 0;
+      for (int c = 0; c < S; ++c) {
+        const float part = __shfl_sync(0xFFFFFFFFu, use_p ? pp : rp, c);
+        if (part > 0.f) { clast = c; prelast = run; }
+        if (cstar < 0 && run + part > t) { cstar = c; pre = run; }
+        run += part;
+      }
+      if (cstar < 0) { cstar = clast; pre = prelast; }
+      const unsigned anyto = __ballot_sync(0xFFFFFFFFu, to != 0);
+      if (lane == 0) {
+        sm.cstar = cstar;
+        sm.tl = t - pre;
+        sm.total = total;
+        sm.use_p = use_p;
+        sm.tmo = anyto ? 1 : 0;
+      }
+    }
+    __syncthreads();
+    if (warp == 0) {
+      const int s_star = sm.cstar;
+      const bool use_p = sm.use_p != 0;
+      const DrawPart* dp = &dparts[s_star];
+      const int e0s = s_star * a.chunk;
+      const int e1s = min(V, e0s + a.chunk);
+      const int nvs = (max(0, e1s - e0s) + VE - 1) / VE;
+      const int nchs = (nvs + kChunkVecs - 1) / kChunkVecs;
+      const float tl = sm.tl;
+      // chunk level: lane c holds chunk c's total
+      float my = 0.f;
+      if (lane < nchs) {
+        for (int w = 0; w < kWarps; ++w) my += use_p ? __ldcg(&dp->ps[lane][w]) : __ldcg(&dp->rs[lane][w]);
+      }
+      float run = 0.f, pre_k = 0.f, pre_last = 0.f;
+      int k_star = -1, k_last = 0;
+      for (int c = 0; c < nchs; ++c) {
+        const float tk = __shfl_sync(0xFFFFFFFFu, my, c);
+        if (tk > 0.f) { k_last = c; pre_last = run; }
+        if (k_star < 0 && run + tk > tl) { k_star = c; pre_k = run; }
+        run += tk;
+      }
+      if (k_star < 0) { k_star = k_last; pre_k = pre_last; }
+      const float tl2 = tl - pre_k;
+      float mw = 0.f;
+      if (lane < kWarps) mw = use_p ? __ldcg(&dp->ps[k_star][lane]) : __ldcg(&dp->rs[k_star][lane]);
+      run = 0.f;
+      float pre_w = 0.f;
+      pre_last = 0.f;
+      int w_star = -1, w_last = 0;
+      for (int w = 0; w < kWarps; ++w) {
+        const float tw = __shfl_sync(0xFFFFFFFFu, mw, w);
+        if (tw > 0.f) { w_last = w; pre_last = run; }
+        if (w_star < 0 && run + tw > tl2) { w_star = w; pre_w = run; }
+        run += tw;
+      }
+      if (w_star < 0) { w_star = w_last; pre_w = pre_last; }
+      const float tl3 = tl2 - pre_w;
+      // lane level: the 32 vectors of that warp in that chunk, re-read from L2
+      const int g = k_star * kChunkVecs + w_star * 32 + lane;
+      float val[VE], pv[VE];
+      if (g < nvs) {
+        draw_vals<TIn, kAligned>(draw, baseP, rbP, baseQ, rbQ, e0s, e1s, g, nullptr, nullptr, cT, nmP, nmQ, invSP, wS,
+                                 wN, check_S, st.bx, st.bi, use_p, val, pv);
+      } else {
+#pragma unroll
+        for (int i = 0; i < VE; ++i) val[i] = 0.f;
+      }
+      float ls = 0.f;
+#pragma unroll
+      for (int i = 0; i < VE; ++i) ls += val[i];
+      float incl = ls;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const float y = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      const unsigned cross = __ballot_sync(0xFFFFFFFFu, incl > tl3);
+      const unsigned pos = __ballot_sync(0xFFFFFFFFu, ls > 0.f);
+      const int l_star = cross ? (__ffs(cross) - 1) : (pos ? (31 - __clz(pos)) : 0);
+      if (lane == l_star) {
+        const float tl4 = tl3 - (incl - ls);
+        float run4 = 0.f, c_prev = 0.f, c_prev_last = 0.f;
+        int i_star = -1, i_last = 0;
+        for (int i = 0; i < VE; ++i) {
+          if (val[i] > 0.f) { i_last = i; c_prev_last = run4; }
+          if (i_star < 0 && run4 + val[i] > tl4) { i_star = i; c_prev = run4; }
+          run4 += val[i];
+        }
+        if (i_star < 0) { i_star = i_last; c_prev = c_prev_last; }
+        const int v = e0s + g * VE + i_star;
+        const float lo = tl4 - c_prev;                // t - CDF before v
+        const float hi = c_prev + val[i_star] - tl4;  // CDF at v - t
+        sm.drawn = min(max(v, 0), V - 1);
+        sm.margin = fminf(fabsf(lo), fabsf(hi)) / sm.total;
+      }
+    }
+    __syncthreads();
+    if (tid == 0) a.draw_arrive[du] = 0;
+  } else {
+    // No stream: greedy (the argmax is the draw) or an invalid row.
+    if (tid == 0) {
+      sm.drawn = row_invalid ? -1 : (verify ? st.argP : st.argQ);
+      sm.margin = INFINITY;
+      sm.total = 1.f;
+      sm.use_p = 0;
+      sm.tmo = 0;
+    }
+    __syncthreads();
+  }
+  if (tid == 0 && (a.F != nullptr || a.alpha != nullptr)) load_plan(a, b, sm.s_F);
+  __syncthreads();
+
+  // ============ finishing the row (verify) or the draft position (reweight) ===========
+  const bool tmo_all = sm.tmo != 0;
+  if (!verify) {
+    if (tid == 0) {
+      const bool ok = !row_invalid && !tmo_all;
+      a.draft_tokens[static_cast<long long>(b) * K + j] = ok ? sm.drawn : -1;
+      UnitState* us = a.ustate + u;
+      us->dmargin = sm.margin;
+      if (tmo_all) us->flags = st.flags | kFlagTimeout;
+      __threadfence();
+      sm.is_last_row = atomicAdd(a.row_arrive2 + b, 1) == K - 1;
+      if (sm.is_last_row) {
+        __threadfence();
+        int fl = a.rstate[b].flags;
+        for (int k = 0; k < K; ++k) {
+          const UnitState* uk = a.ustate + static_cast<long long>(b) * (K + 1) + k;
+          fl |= __ldcg(&uk->flags);
+          if (__ldcg(&uk->dmargin) < kNearTie) fl |= SSD_ROW_NEAR_TIE;
+        }
+        a.status[b] = fl;
+        a.row_arrive2[b] = 0;
+      }
+    }
+    return;
+  }
+
+  const int kstar = j;
+  int fl = rowflags | (tmo_all ? kFlagTimeout : 0);
+  const bool invalid = (fl & SSD_ROW_INVALID) != 0;
+  if (tid == 0) {
+    if (!kGreedy && (amargin < kNearTie || sm.margin < kNearTie)) fl |= SSD_ROW_NEAR_TIE;
+    fl &= ~SSD_ROW_ZERO_RESIDUAL;
+    if (sm.use_p) fl |= SSD_ROW_ZERO_RESIDUAL;
+    a.status[b] = fl;
+    a.n_accepted[b] = invalid ? -1 : kstar;
+    a.bonus[b] = invalid ? -1 : sm.drawn;
+    a.residual_mass[b] = invalid ? __int_as_float(0x7FC00000) : sm.total;
+    sm.slot = -1;
+  }
+  if (tid <= K) {
+    int32_t t = -1;
+    if (!invalid) t = tid < kstar ? __ldg(a.tokens + static_cast<long long>(b) * K + tid) : (tid == kstar ? sm.drawn : -1);
+    a.out_tokens[static_cast<long long>(b) * (K + 1) + tid] = t;
+  }
+  if (invalid)
+    for (int k = tid; k < K; k += kThreads) a.accept_prob[static_cast<long long>(b) * K + k] = __int_as_float(0x7FC00000);
+  if (a.c_tokens) {
+    const bool pbad = (fl & SSD_ROW_BAD_PLAN) != 0;
+    if (tid == 0) {
+      int off = 0;
+      a.c_offsets[static_cast<long long>(b) * (K + 2)] = 0;
+      for (int k = 0; k <= K; ++k) {
+        off += pbad ? 0 : sm.s_F[k];
+        a.c_offsets[static_cast<long long>(b) * (K + 2) + k + 1] = off;
+      }
+    }
+    __syncthreads();
+    if (invalid) {
+      for (int s2 = tid; s2 < a.budget; s2 += kThreads) a.c_tokens[static_cast<long long>(b) * a.budget + s2] = -1;
+    } else {
+      // the key (k*, bonus) in segment k* of the row's cache
+      int off = 0;
+      for (int k = 0; k < kstar; ++k) off += sm.s_F[k];
+      const int32_t* seg = a.c_tokens + static_cast<long long>(b) * a.budget + off;
+      for (int i = tid; i < sm.s_F[kstar]; i += kThreads)
+        if (__ldcg(seg + i) == sm.drawn) sm.slot = off + i;
+    }
+    __syncthreads();
+    const int slot = sm.slot;
+    if (tid == 0) {
+      a.c_hit[b] = slot >= 0 ? 1 : 0;
+      a.c_slot[b] = slot;
+    }
+    for (int i = tid; i < K; i += kThreads) {
+      int32_t t;
+      if (slot >= 0)
+        t = a.c_payload ? __ldg(a.c_payload + (static_cast<long long>(b) * a.budget + slot) * K + i) : -1;
+      else
+        t = fallback_token(a.fallback_seed, b, i, V);
+      a.c_next[static_cast<long long>(b) * K + i] = t;
+    }
+  }
+}
+
+}  // namespace ssd

@@ -37,9 +37,13 @@ def test_status_strings_and_version():
 
 
 def test_workspace_size_formula():
-    assert ssd.workspace_bytes(64, 6) % 256 == 0
-    assert ssd.workspace_bytes(64, 6) >= 64 * 7 * 32 + 64 * 8 + 4
-    assert ssd.load().ssd_workspace_bytes(1, 0, 10, 1) == 0
+    n = ssd.workspace_bytes(64, 6, 128256, ssd.DTYPE_BF16)
+    assert n % 256 == 0 and n >= 64 * 7 * 8 * 1056
+    assert ssd.workspace_bytes(64, 6, 128256, ssd.DTYPE_BF16) <= ssd.workspace_bytes(64, 6, 262144, ssd.DTYPE_BF16)
+    L = ssd.load()
+    assert L.ssd_workspace_bytes(1, 0, 10, 1) == 0
+    assert L.ssd_workspace_bytes(1, 2, 0, 1) == 0
+    assert L.ssd_workspace_bytes(1, 2, 10, 9) == 0
 
 
 def test_host_validation_without_gpu():
