@@ -159,6 +159,36 @@ ssd_status ssd_verify(const void* target_logits, const void* draft_logits, const
                       int32_t* status, void* workspace, size_t ws_bytes, void* stream);
 
 /*
+ * ssd_verify_noalloc -- ssd_verify with its scratch taken from a static
+ * device buffer of this library instead of a caller-provided workspace.  The
+ * pages describe no such call: it exists for callers that cannot allocate
+ * device memory at the moment they verify -- a serving loop that handed
+ * every byte of HBM to its KV cache at start-up, a host program with no
+ * device allocator of its own, or code that must not let cudaMalloc/cudaFree
+ * synchronise the device in the middle of a decode step.  It calls no
+ * allocating function (no cudaMalloc, cudaFree or library allocation).
+ *   Arguments, layouts, outputs and row status: exactly as ssd_verify, minus
+ *   workspace and ws_bytes.
+ *   Limit: the problem's ssd_workspace_bytes(B, K, V, dtype) must not exceed
+ *   SSD_NOALLOC_MAX_WORKSPACE (16 MiB, enough for B=64, K=6, V=128256 bf16);
+ *   larger problems return SSD_ERR_WORKSPACE before touching the device.
+ *   First call on a device: looks up the buffer's device address
+ *   (cudaGetSymbolAddress, with that device current) and zero-fills it with a
+ *   synchronous memset; make that first call before any stream capture.
+ *   Later calls only launch.  The buffer is one per device: calls that
+ *   overlap on one device (two streams, or two host threads) share it and
+ *   race; serialise them.  Each completed call leaves its counters zero.
+ */
+#define SSD_NOALLOC_MAX_WORKSPACE (16u << 20)
+ssd_status ssd_verify_noalloc(const void* target_logits, const void* draft_logits, const void* draft_next,
+                              int dtype, int B, int K, int V, const int32_t* draft_tokens,
+                              const float* uniforms, float T, const int32_t* F, const float* alpha,
+                              int fanout_mode, float C, int budget,
+                              int32_t* n_accepted, int32_t* bonus, int32_t* out_tokens,
+                              float* accept_prob, float* residual_mass, const ssd_cache* cache,
+                              int32_t* status, void* stream);
+
+/*
  * ssd_cache_build -- pack per-outcome guess lists into the cache layout
  * ([ZH] section 2, basic flow step 3).  offsets[b] = prefix sums of F[b];
  * tokens[b, offsets[b,k] + i] = topf_tokens[b, offsets[b,k] + i] for k < K

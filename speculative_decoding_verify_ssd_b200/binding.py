@@ -79,6 +79,9 @@ def load(build_if_missing: bool = True):
     L.ssd_verify.restype = i32
     L.ssd_verify.argtypes = [vp, vp, vp, i32, i32, i32, i32, vp, vp, f32, vp, vp, i32, f32, i32, vp, vp,
                              vp, vp, vp, C.POINTER(_Cache), vp, vp, sz, vp]
+    L.ssd_verify_noalloc.restype = i32
+    L.ssd_verify_noalloc.argtypes = [vp, vp, vp, i32, i32, i32, i32, vp, vp, f32, vp, vp, i32, f32, i32, vp, vp,
+                                     vp, vp, vp, C.POINTER(_Cache), vp, vp]
     L.ssd_cache_build.restype = i32
     L.ssd_cache_build.argtypes = [vp, vp, vp, i32, i32, i32, vp, vp, vp]
     L.ssd_cache_lookup.restype = i32
@@ -245,6 +248,54 @@ def ssd_verify(target: torch.Tensor, draft: torch.Tensor, draft_tokens: torch.Te
         C.byref(cstruct) if cstruct is not None else None, _ptr(out.status), workspace.ptr(),
         workspace.nbytes, _stream(stream))
     _check(code, "ssd_verify")
+    return out
+
+
+NOALLOC_MAX_WORKSPACE = 16 << 20
+
+
+def ssd_verify_noalloc(target: torch.Tensor, draft: torch.Tensor, draft_tokens: torch.Tensor,
+                       uniforms: torch.Tensor, T: float, out: VerifyResult, F: Optional[torch.Tensor] = None,
+                       C_coef: float = 1.0, budget: int = 0, draft_next: Optional[torch.Tensor] = None,
+                       cache: bool = False, alpha: Optional[torch.Tensor] = None,
+                       fanout_mode: int = FANOUT_GEOMETRIC, payload: Optional[torch.Tensor] = None,
+                       fallback_seed: int = 0, stream=None) -> VerifyResult:
+    """ssd_verify with the library's static scratch instead of a workspace
+    (see ssd_verify_noalloc in ssd.h).  The caller passes `out` (from
+    alloc_verify_result, made once ahead of time), so the call itself makes no
+    device allocation.  Calls on one device must not overlap."""
+    B, K1, V = target.shape
+    K = K1 - 1
+    dev = target.device
+    if dev.type != "cuda":
+        raise ValueError("ssd_verify_noalloc runs on a CUDA device")
+    dt = _logit_dtype(target)
+    _need(target, "target", target.dtype, (B, K + 1, V), dev)
+    _need(draft, "draft", target.dtype, (B, K, V), dev)
+    if draft_next is not None:
+        _need(draft_next, "draft_next", target.dtype, (B, V), dev)
+    _need(draft_tokens, "draft_tokens", torch.int32, (B, K), dev)
+    _need(uniforms, "uniforms", torch.float32, (B, K + 1), dev)
+    if F is not None:
+        _need(F, "F", torch.int32, (B, K + 1), dev)
+    if alpha is not None:
+        _need(alpha, "alpha", torch.float32, (B,), dev)
+    if payload is not None:
+        _need(payload, "payload", torch.int32, (B, budget, K), dev)
+    if cache and F is None and alpha is None:
+        raise ValueError("a cache needs a fan-out plan (F or alpha)")
+    cstruct = None
+    if cache:
+        cstruct = _Cache(out.cache_offsets.data_ptr(), out.cache_tokens.data_ptr(),
+                         None if payload is None else payload.data_ptr(), out.hit.data_ptr(),
+                         out.slot.data_ptr(), out.next_tokens.data_ptr(), fallback_seed)
+    code = load().ssd_verify_noalloc(
+        _ptr(target), _ptr(draft), _ptr(draft_next), dt, B, K, V, _ptr(draft_tokens), _ptr(uniforms),
+        float(T), _ptr(F), _ptr(alpha), int(fanout_mode), float(C_coef), int(budget),
+        _ptr(out.n_accepted), _ptr(out.bonus),
+        _ptr(out.out_tokens), _ptr(out.accept_prob), _ptr(out.residual_mass),
+        C.byref(cstruct) if cstruct is not None else None, _ptr(out.status), _stream(stream))
+    _check(code, "ssd_verify_noalloc")
     return out
 
 

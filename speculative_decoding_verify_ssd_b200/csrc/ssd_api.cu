@@ -420,3 +420,50 @@ ssd_status ssd_saguaro_reweight(const void* draft_logits, int dtype, int B, int 
 }
 
 }  // extern "C"
+
+// ---- ssd_verify_noalloc: the scratch in a static device buffer -------------------
+// For callers that cannot allocate device memory when they verify (a server
+// whose HBM is all handed out at start-up, a host program without a device
+// allocator, code that must not let cudaMalloc/cudaFree synchronise the
+// device).  The buffer is this module's own static device memory; nothing
+// here calls an allocating function.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[SSD_NOALLOC_MAX_WORKSPACE];
+static constexpr int kNoallocMaxDevices = 64;
+static void* g_noalloc_ptr[kNoallocMaxDevices];
+static std::mutex g_noalloc_mu;
+
+// The buffer's address on the current device; the first call per device also
+// zero-fills it (the arrival counters must start at zero) and waits for that.
+static ssd_status noalloc_scratch(void** out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kNoallocMaxDevices) return SSD_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return SSD_ERR_CUDA;
+    if (cudaMemset(p, 0, SSD_NOALLOC_MAX_WORKSPACE) != cudaSuccess) return SSD_ERR_CUDA;
+    if (cudaDeviceSynchronize() != cudaSuccess) return SSD_ERR_CUDA;
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return SSD_OK;
+}
+
+extern "C" ssd_status ssd_verify_noalloc(const void* target_logits, const void* draft_logits, const void* draft_next,
+                                         int dtype, int B, int K, int V, const int32_t* draft_tokens,
+                                         const float* uniforms, float T, const int32_t* F, const float* alpha,
+                                         int fanout_mode, float C, int budget, int32_t* n_accepted, int32_t* bonus,
+                                         int32_t* out_tokens, float* accept_prob, float* residual_mass,
+                                         const ssd_cache* cache, int32_t* status, void* stream) {
+  if (dtype != SSD_DTYPE_BF16 && dtype != SSD_DTYPE_FP32) return SSD_ERR_DTYPE;
+  if (B < 0 || K < 1 || K > SSD_MAX_K || V < 1) return SSD_ERR_INVALID_ARG;
+  if (ssd_workspace_bytes(B, K, V, dtype) > SSD_NOALLOC_MAX_WORKSPACE) return SSD_ERR_WORKSPACE;
+  void* scratch = nullptr;
+  if (B > 0) {
+    const ssd_status s = noalloc_scratch(&scratch);
+    if (s != SSD_OK) return s;
+  }
+  return ssd_verify(target_logits, draft_logits, draft_next, dtype, B, K, V, draft_tokens, uniforms, T, F, alpha,
+                    fanout_mode, C, budget, n_accepted, bonus, out_tokens, accept_prob, residual_mass, cache, status,
+                    scratch, SSD_NOALLOC_MAX_WORKSPACE, stream);
+}
