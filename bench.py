@@ -130,6 +130,32 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
+def rank_workload(w, rank):
+    """Rank `rank`'s share under weak scaling: the same workload shape with
+    its own seeds, so every rank verifies different rows."""
+    return w.replace(seed=w.seed + 7919 * rank, fallback_seed=w.fallback_seed + rank)
+
+
+def max_over_ranks(value, dist, device):
+    """The slowest rank's time: one all-reduce (MAX) of a scalar, taken by
+    every rank at the same point."""
+    import torch
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_rows_per_s(world, B, steps, max_ms):
+    """Whole-job throughput: rows verified by all ranks over the slowest rank's time."""
+    return world * B * steps / (max_ms / 1e3)
+
+
+def workload_config(w, world):
+    return {"workload": w.name, "B": w.B, "K": w.K, "V": w.V, "T": w.T, "budget": w.budget, "C": w.C,
+            "fanout": "geometric" if w.fanout_mode == 0 else "uniform", "alpha": w.alpha,
+            "parallelism": f"rows sharded, {world} independent GPU(s)"}
+
+
 def algorithmic_bytes(w):
     s = 2 if w.dtype == "bf16" else 4
     logits = w.B * (2 * w.K + 1) * w.V * s
@@ -148,7 +174,7 @@ def run_ssd(args, rank, world, local_rank):
     torch.cuda.set_device(dev)
     ssd.load()
     w = synth.WORKLOADS[args.workload]
-    w_rank = w.replace(seed=w.seed + 7919 * rank, fallback_seed=w.fallback_seed + rank)
+    w_rank = rank_workload(w, rank)
     logit_bytes, alg_bytes = algorithmic_bytes(w)
     n_copies = max(2, -(-2 * L2_BYTES // logit_bytes))
     n_copies = min(n_copies, 8)
@@ -233,11 +259,9 @@ def run_ssd(args, rank, world, local_rank):
     # the graph holds `steps` verify calls back to back: per-step time = replay time / steps
     kernel_ms = [a.elapsed_time(b) / args.steps for a, b in per_rep]
     if world > 1:
-        t = torch.tensor([total_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+        total_ms = max_over_ranks(total_ms, dist, dev)
     ms_per_step = total_ms / steps_done
-    rows_per_s = world * w.B * steps_done / (total_ms / 1e3)
+    rows_per_s = job_rows_per_s(world, w.B, steps_done, total_ms)
     del graph
 
     # outcome statistics from the last step of each rotating copy
@@ -324,7 +348,7 @@ def run_reference(args, rank, world):
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "rows/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * t_all / max(1, args.steps),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic", "config": {"workload": w.name, "B": w.B, "K": w.K, "V": w.V},
+            "data": "synthetic", "config": workload_config(w, world),
             "cpu_baseline": {"value": value, "unit": "rows/s", "cores": cores, "kind": "oracle",
                              "sample": f"{cores} rows of {w.name} per step"},
             "e2e": {"value": value, "unit": "rows/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -390,11 +414,9 @@ def main():
         "vs_baseline": None,
         "dtype": w.dtype,
         "data": "synthetic",
-        "config": {"workload": w.name, "B": w.B, "K": w.K, "V": w.V, "T": w.T, "budget": w.budget, "C": w.C,
-                   "fanout": "geometric" if w.fanout_mode == 0 else "uniform", "alpha": w.alpha,
-                   "parallelism": f"rows sharded, {world} independent GPU(s)",
-                   "l2": f"{res['n_copies']} rotating input copies of {res['logit_bytes'] / 1e6:.1f} MB "
-                         f"(each > 126 MB L2)"},
+        "config": dict(workload_config(w, world),
+                       l2=f"{res['n_copies']} rotating input copies of {res['logit_bytes'] / 1e6:.1f} MB "
+                          f"(each > 126 MB L2)"),
         "hbm_gbs": achieved,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "traffic": traffic,
