@@ -102,7 +102,7 @@ __global__ void cache_lookup_kernel(const int32_t* __restrict__ offsets, const i
 // Launch planning.
 // ---------------------------------------------------------------------------
 #ifndef SSD_CTA_BYTES
-#define SSD_CTA_BYTES 65536   // logits streamed per CTA (all rows of a unit slice)
+#define SSD_CTA_BYTES 131072  // logits streamed per CTA (all rows of a unit slice)
 #endif
 constexpr long long kCtaBytes = SSD_CTA_BYTES;
 constexpr int kMinChunk = 1024;  // do not split a row finer than this

@@ -487,13 +487,83 @@ __device__ __forceinline__ void unit_rows(const Args& a, int b, int j, const TIn
   }
 }
 
-// The row's fan-out plan into shared memory (thread 0): F when given, else
-// planned from alpha.  Returns nothing; callers check Σ F = budget, 0 <= F <= V.
-__device__ __forceinline__ void load_plan(const Args& a, int b, int32_t* s_F) {
+// The same plan on one warp: lane k holds F_k in f[0] and F_{k+32} in f[1].
+// Lane k forms alpha^k by k rounded products, so every quota, remainder and
+// tie equals the serial one; the repeated largest-remainder picks become a
+// rank: a lane of rank r among the remainders (larger first, ties to the
+// smaller k) gets rem / (K+1) + (r < rem % (K+1)) extra seats.
+__device__ __forceinline__ void fanout_warp(float alpha_f, int K, int budget, int mode, int lane, int (&f)[2]) {
+  const int n = K + 1;
+  f[0] = f[1] = 0;
+  if (mode == SSD_FANOUT_UNIFORM) {
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int k = lane + 32 * h;
+      if (k < n) f[h] = budget / n + (k < budget % n ? 1 : 0);
+    }
+    return;
+  }
+  const double al = static_cast<double>(alpha_f);
+  if (!(al >= 0.0 && al <= 1.0)) {
+    if (lane == 0) f[0] = -1;
+    return;
+  }
+  double frac[2] = {0.0, 0.0};
+  int assigned = 0;
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const int k = lane + 32 * h;
+    if (k < n) {
+      double run = 1.0;
+      for (int i = 0; i < k; ++i) run = __dmul_rn(run, al);
+      const double P = k < K ? __dmul_rn(run, __dsub_rn(1.0, al)) : run;
+      const double quota = __dmul_rn(static_cast<double>(budget), P);
+      const double fl = floor(quota);
+      f[h] = static_cast<int>(fl);
+      frac[h] = __dsub_rn(quota, fl);
+      assigned += f[h];
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) assigned += __shfl_xor_sync(0xFFFFFFFFu, assigned, o);
+  const int rem = budget - assigned;
+  if (rem <= 0) return;
+  int rank[2] = {0, 0};
+  for (int i = 0; i < n; ++i) {
+    const double src = i < 32 ? frac[0] : frac[1];
+    const double fi = __shfl_sync(0xFFFFFFFFu, src, i & 31);
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int k = lane + 32 * h;
+      if (k < n && i != k && (fi > frac[h] || (fi == frac[h] && i < k))) ++rank[h];
+    }
+  }
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const int k = lane + 32 * h;
+    if (k < n) f[h] += rem / n + (rank[h] < rem % n ? 1 : 0);
+  }
+}
+
+// The row's fan-out plan into shared memory, by one whole warp: F when
+// given, else planned from alpha.  Callers check Σ F = budget, 0 <= F <= V.
+__device__ __forceinline__ void load_plan(const Args& a, int b, int32_t* s_F, int lane) {
+  const int n = a.K + 1;
+  int f[2] = {0, 0};
   if (a.F) {
-    for (int k = 0; k <= a.K; ++k) s_F[k] = __ldg(a.F + static_cast<long long>(b) * (a.K + 1) + k);
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int k = lane + 32 * h;
+      if (k < n) f[h] = __ldg(a.F + static_cast<long long>(b) * n + k);
+    }
   } else {
-    fanout_row(__ldg(a.alpha + b), a.K, a.budget, a.fanout_mode, s_F);
+    const float al = a.fanout_mode == SSD_FANOUT_UNIFORM ? 0.f : __ldg(a.alpha + b);
+    fanout_warp(al, a.K, a.budget, a.fanout_mode, lane, f);
+  }
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const int k = lane + 32 * h;
+    if (k < n) s_F[k] = f[h];
   }
 }
 
@@ -553,7 +623,7 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) ssd_stats_kernel(const _
   if constexpr (kAligned) ring.start(tid);
 
   const bool has_plan = a.F != nullptr || a.alpha != nullptr;
-  if (tid == 0 && has_plan) load_plan(a, b, sm.s_F);
+  if (warp == 0 && has_plan) load_plan(a, b, sm.s_F, lane);
   int flags = 0, d = -1;
   float u_self = 0.f;
   if (has_d) {
@@ -587,9 +657,9 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) ssd_stats_kernel(const _
   // ---- the stream: online max / exp-sum (or greedy argmax) of both rows ----------
   float mP = -INFINITY, sP = 0.f, nmP1 = 0.f, mQ = -INFINITY, sQ = 0.f, nmQ1 = 0.f;
   int argP = INT_MAX, argQ = INT_MAX, nan_seen = 0, tmo = 0;
-  float vm1 = -INFINITY, vm2 = -INFINITY;  // top two vector maxima of the source row
-  int g1 = -1;
-  uint4 keep = make_uint4(0u, 0u, 0u, 0u);  // the source vector holding vm1
+  float vm1 = -INFINITY, vm2 = -INFINITY, vm3 = -INFINITY;  // top three vector maxima of the source row
+  int g1 = -1, g2 = -1;
+  uint4 keep1 = make_uint4(0u, 0u, 0u, 0u), keep2 = keep1;  // the source vectors holding vm1, vm2
   for (int c = 0; c < nch; ++c) {
     if constexpr (kAligned) ring.acquire(c, tid, tmo);
     const int g = c * kChunkVecs + tid;
@@ -622,9 +692,14 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) ssd_stats_kernel(const _
         vsrc = srcQ ? vq : vp;
         wsrc = srcQ ? wq : wp;
       }
-      if (vsrc > vm2) {
-        if (vsrc > vm1) { vm2 = vm1; vm1 = vsrc; g1 = g; keep = wsrc; }
-        else vm2 = vsrc;
+      if (vsrc > vm3) {
+        if (vsrc > vm2) {
+          vm3 = vm2;
+          if (vsrc > vm1) { vm2 = vm1; keep2 = keep1; g2 = g1; vm1 = vsrc; g1 = g; keep1 = wsrc; }
+          else { vm2 = vsrc; g2 = g; keep2 = wsrc; }
+        } else {
+          vm3 = vsrc;
+        }
       }
     }
   }
@@ -697,18 +772,29 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) ssd_stats_kernel(const _
   __syncthreads();
   const float tau = sm.tau;
 
-  // Local candidates: the elements at or above tau.  A thread whose second
-  // vector maximum is below tau holds them all in its kept vector.
+  // Local candidates: the elements at or above tau.  A thread whose third
+  // vector maximum is below tau holds them all in its two kept vectors.
   if (fast_ok && vm1 >= tau && vm1 == vm1) {
-    if (kAligned && vm2 < tau) {
+    if (kAligned && vm3 < tau) {
       float x[VE];
-      Elem<TIn>::unpack(keep, x);
+      Elem<TIn>::unpack(keep1, x);
 #pragma unroll
       for (int i = 0; i < VE; ++i) {
         const int v = e0 + g1 * VE + i;
         if (x[i] >= tau && v < e1) {
           const int pos = atomicAdd(&sm.n_raw, 1);
           if (pos < kCandCap) sm.raw[pos] = Cand{x[i], v};
+        }
+      }
+      if (vm2 >= tau && g2 >= 0) {
+        Elem<TIn>::unpack(keep2, x);
+#pragma unroll
+        for (int i = 0; i < VE; ++i) {
+          const int v = e0 + g2 * VE + i;
+          if (x[i] >= tau && v < e1) {
+            const int pos = atomicAdd(&sm.n_raw, 1);
+            if (pos < kCandCap) sm.raw[pos] = Cand{x[i], v};
+          }
         }
       }
     } else {
@@ -1238,7 +1324,7 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) ssd_draw_kernel(const __
     }
     __syncthreads();
   }
-  if (tid == 0 && (a.F != nullptr || a.alpha != nullptr)) load_plan(a, b, sm.s_F);
+  if (warp == 0 && (a.F != nullptr || a.alpha != nullptr)) load_plan(a, b, sm.s_F, lane);
   __syncthreads();
 
   // ============ finishing the row (verify) or the draft position (reweight) ===========
