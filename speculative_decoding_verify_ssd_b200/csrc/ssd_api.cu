@@ -105,6 +105,10 @@ __global__ void cache_lookup_kernel(const int32_t* __restrict__ offsets, const i
 #define SSD_CTA_BYTES 131072  // logits streamed per CTA (all rows of a unit slice)
 #endif
 constexpr long long kCtaBytes = SSD_CTA_BYTES;
+#ifndef SSD_DRAW_CTA_BYTES
+#define SSD_DRAW_CTA_BYTES 32768  // logits streamed per CTA of the draw kernel
+#endif
+constexpr long long kDrawCtaBytes = SSD_DRAW_CTA_BYTES;
 constexpr int kMinChunk = 1024;  // do not split a row finer than this
 
 struct Plan {
@@ -118,16 +122,18 @@ static int sm_count() {
 }
 
 // Slices per logit row and the slice length, for units of `rows` rows of length V.
-static ssd_status make_plan(int V, int rows, int esize, long long units, Plan* p) {
+static ssd_status make_plan(int V, int rows, int esize, long long units, Plan* p,
+                            long long cta_bytes = kCtaBytes) {
   const int VE = 16 / esize;
   const long long max_chunk = static_cast<long long>(kMaxChunks) * kChunkVecs * VE;
-  long long ns = (static_cast<long long>(rows) * V * esize + kCtaBytes - 1) / kCtaBytes;
+  long long ns = (static_cast<long long>(rows) * V * esize + cta_bytes - 1) / cta_bytes;
   // enough CTAs to fill the machine, if the rows are long enough
   const long long want = (static_cast<long long>(kMinBlocks) * sm_count() + units - 1) / (units > 0 ? units : 1);
   const long long by_len = (V + kMinChunk - 1) / kMinChunk;
   long long extra = want < by_len ? want : by_len;
   if (extra > 8) extra = 8;
   if (ns < extra) ns = extra;
+  if (ns > kMaxSlices) ns = kMaxSlices;
   if (ns < 1) ns = 1;
   long long chunk = (V + ns - 1) / ns;
   chunk = (chunk + VE - 1) / VE * VE;
@@ -173,6 +179,9 @@ static int plan_slices(int B, int K, int V, int dtype) {
   int ns = 1;
   if (make_plan(V, 2, esize, units, &p2) == SSD_OK) ns = p2.n_slices;
   if (make_plan(V, 1, esize, units, &p1) == SSD_OK) ns = ns > p1.n_slices ? ns : p1.n_slices;
+  if (make_plan(V, 2, esize, B, &p2, kDrawCtaBytes) == SSD_OK) ns = ns > p2.n_slices ? ns : p2.n_slices;
+  if (make_plan(V, 1, esize, static_cast<long long>(B) * K, &p1, kDrawCtaBytes) == SSD_OK)
+    ns = ns > p1.n_slices ? ns : p1.n_slices;
   return ns;
 }
 
@@ -216,13 +225,13 @@ static ssd_status launch_t(const Args& a, long long units, long long draw_units,
   const void* f1 = reinterpret_cast<const void*>(&ssd_stats_kernel<TIn, kAligned, kGreedy>);
   const void* f2 = reinterpret_cast<const void*>(&ssd_draw_kernel<TIn, kAligned, kGreedy>);
   if (prepare_kernel(f1) != cudaSuccess || prepare_kernel(f2) != cudaSuccess) return SSD_ERR_CUDA;
-  const size_t smem = kAligned ? kRingBytes : 0;
+  const size_t smem = kRingBytes;  // the ring, and afterwards the merge buffers
   ssd_stats_kernel<TIn, kAligned, kGreedy>
       <<<static_cast<unsigned>(units * a.n_slices), kThreads, smem, stream>>>(a);
   if (cudaGetLastError() != cudaSuccess) return SSD_ERR_CUDA;
   if (draw_units > 0) {
     ssd_draw_kernel<TIn, kAligned, kGreedy>
-        <<<static_cast<unsigned>(draw_units * a.n_slices), kThreads, smem, stream>>>(a);
+        <<<static_cast<unsigned>(draw_units * a.d_slices), kThreads, smem, stream>>>(a);
     if (cudaGetLastError() != cudaSuccess) return SSD_ERR_CUDA;
   }
   return SSD_OK;
@@ -361,6 +370,11 @@ ssd_status ssd_verify(const void* target_logits, const void* draft_logits, const
   a.fanout_mode = fanout_mode;
   a.B = B; a.K = K; a.V = V; a.budget = budget; a.mode = kModeVerify;
   a.n_slices = plan.n_slices; a.chunk = plan.chunk; a.units_per_row = K + 1; a.draws = 1;
+  Plan dplan;
+  const ssd_status dps = make_plan(V, 2, esize, B, &dplan, kDrawCtaBytes);
+  if (dps != SSD_OK) return dps;
+  if (dplan.n_slices > wl.n_slices) return SSD_ERR_WORKSPACE;
+  a.d_slices = dplan.n_slices; a.d_chunk = dplan.chunk;
   a.T = T; a.C = has_plan ? C : 1.f;
   a.n_accepted = n_accepted; a.bonus = bonus; a.out_tokens = out_tokens; a.accept_prob = accept_prob;
   a.residual_mass = residual_mass; a.status = status;
@@ -407,6 +421,11 @@ ssd_status ssd_saguaro_reweight(const void* draft_logits, int dtype, int B, int 
   a.F = F;
   a.B = B; a.K = K; a.V = V; a.budget = budget; a.mode = kModeReweight;
   a.n_slices = plan.n_slices; a.chunk = plan.chunk; a.units_per_row = per_row;
+  Plan dplan;
+  const ssd_status dps = make_plan(V, 1, esize, static_cast<long long>(B) * K, &dplan, kDrawCtaBytes);
+  if (dps != SSD_OK) return dps;
+  if (dplan.n_slices > wl.n_slices) return SSD_ERR_WORKSPACE;
+  a.d_slices = dplan.n_slices; a.d_chunk = dplan.chunk;
   a.T = T; a.C = C;
   a.status = status;
   a.topf_tokens = topf_tokens; a.offsets = offsets; a.Z = Z; a.q_lse = q_lse; a.draft_tokens = draft_tokens_out;

@@ -45,7 +45,7 @@ constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
 constexpr int kMinBlocks = 4;          // CTAs per SM the register budget is set for
 constexpr int kMaxSlices = 16;         // slices per logit row
-constexpr int kStages = 4;             // depth of the bulk-copy ring
+constexpr int kStages = 6;             // depth of the bulk-copy ring
 constexpr int kChunkVecs = kThreads;   // 16-byte vectors per row per ring stage
 constexpr int kMaxChunks = 16;         // ring chunks per slice
 constexpr int kCandCap = 256;          // local top-F candidates found by a CTA
@@ -57,6 +57,8 @@ constexpr uint32_t kMaxPolls = 4000000u;  // x ~0.5 us sleep: about 2 s
 constexpr float kNearTie = 1e-5f;
 constexpr int kFlagTimeout = SSD_ROW_DEVICE_TIMEOUT;
 constexpr size_t kRingBytes = static_cast<size_t>(kStages) * 2 * kChunkVecs * 16;
+
+static_assert(8 * (kCandCap + kGatherCap + kSelCap) <= kRingBytes, "merge buffers must fit in the idle ring");
 
 enum Mode : int { kModeVerify = 0, kModeReweight = 1 };
 enum Draw : int { kDrawNone = 0, kDrawResidual = 1, kDrawP = 2, kDrawQ = 3 };
@@ -91,10 +93,15 @@ struct DrawPart {
   float ps[kMaxChunks][kWarps];
 };
 
+// Kernel 1, per row: the decision and (verify) the statistics of unit k*,
+// so that the draw reads one record.
 struct RowState {
   int32_t kstar, flags;
   float amargin;
-  int32_t pad;
+  int32_t Fj;
+  float MP, SP, MQ, SQ;
+  float Z, bx;
+  int32_t bi, argP;
 };
 
 struct Args {
@@ -109,6 +116,7 @@ struct Args {
   const float* alpha;      // [B]: plan computed in-kernel when F is null
   int fanout_mode;
   int B, K, V, budget, mode, n_slices, chunk, units_per_row;
+  int d_slices, d_chunk;   // kernel 2: slices per drawn row and their length
   int draws;               // kernel 2 runs (verify always; reweight: draft tokens drawn)
   float T, C;
   // verify outputs
@@ -578,8 +586,7 @@ struct Smem1 {
   float tau, MP, SP, MQ, SQ, QS, bx;
   int32_t bi, argP, argQ, n_total, slow, tmo, n_raw, is_last, is_last_row, pad;
   int32_t cand_off[kMaxSlices + 1];
-  Cand raw[kCandCap];
-  Cand buf[kGatherCap + kSelCap];  // the unit's gathered candidates, then its sorted top-F
+  int32_t cnt[kMaxSlices];
 };
 
 template <typename TIn, bool kAligned, bool kGreedy>
@@ -623,7 +630,21 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) ssd_stats_kernel(const _
   if constexpr (kAligned) ring.start(tid);
 
   const bool has_plan = a.F != nullptr || a.alpha != nullptr;
-  if (warp == 0 && has_plan) load_plan(a, b, sm.s_F, lane);
+  // The plan's inputs are loaded now; warp 0 forms the plan after the stream
+  // (only the epilogue needs it).
+  int fplan[2] = {0, 0};
+  float alpha_in = 0.f;
+  if (warp == 0 && has_plan) {
+    if (a.F) {
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int k = lane + 32 * h;
+        if (k <= K) fplan[h] = __ldg(a.F + static_cast<long long>(b) * (K + 1) + k);
+      }
+    } else if (a.fanout_mode != SSD_FANOUT_UNIFORM && lane == 0) {
+      alpha_in = __ldg(a.alpha + b);
+    }
+  }
   int flags = 0, d = -1;
   float u_self = 0.f;
   if (has_d) {
@@ -637,21 +658,6 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) ssd_stats_kernel(const _
     const float ud = __ldg(a.uniforms + static_cast<long long>(b) * K + j);
     if (!(ud >= 0.f && ud < 1.f)) flags |= SSD_ROW_BAD_UNIFORM;
   }
-  __syncthreads();
-  int Fj = 0, seg_off = 0, plan_bad = 0;
-  if (has_plan) {
-    long long sum = 0;
-    for (int k = 0; k <= K; ++k) {
-      const int f = sm.s_F[k];
-      if (f < 0 || f > V) plan_bad = 1;
-      if (k < j) seg_off += f;
-      sum += f;
-    }
-    if (sum != a.budget) plan_bad = 1;
-    Fj = plan_bad ? 0 : sm.s_F[j];
-  }
-  if (plan_bad) flags |= SSD_ROW_BAD_PLAN;
-  const bool want_topf = has_plan && Fj > 0;
   const float cT = kGreedy ? 0.f : kLog2e / a.T;
 
   // ---- the stream: online max / exp-sum (or greedy argmax) of both rows ----------
@@ -706,8 +712,20 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) ssd_stats_kernel(const _
   if constexpr (kGreedy) {
     if (nan_seen) { mP = __int_as_float(0x7FC00000); mQ = mP; }
   }
+  if (warp == 0 && has_plan) {
+    if (!a.F) fanout_warp(__shfl_sync(0xFFFFFFFFu, alpha_in, 0), K, a.budget, a.fanout_mode, lane, fplan);
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int k = lane + 32 * h;
+      if (k <= K) sm.s_F[k] = fplan[h];
+    }
+  }
   sm.gmax[tid] = vm1;
   if (tid == 0) sm.n_raw = 0;
+
+  // The ring is idle from here on: the candidate and merge buffers live in it.
+  Cand* const raw = reinterpret_cast<Cand*>(ring_buf);
+  Cand* const gbuf = raw + kCandCap;  // the unit's gathered candidates, then its sorted top-F
 
   // ---- slice reduction: butterfly within each warp, then over the warps ----------
   if constexpr (kGreedy) {
@@ -731,8 +749,22 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) ssd_stats_kernel(const _
       sm.wred[warp][2] = mQ; sm.wred[warp][3] = sQ;
     }
   }
-  const bool fast_ok = want_topf && Fj <= kMaxGroups;
   tmo = __syncthreads_or(tmo);
+  int Fj = 0, seg_off = 0, plan_bad = 0;
+  if (has_plan) {
+    long long sum = 0;
+    for (int k = 0; k <= K; ++k) {
+      const int f = sm.s_F[k];
+      if (f < 0 || f > V) plan_bad = 1;
+      if (k < j) seg_off += f;
+      sum += f;
+    }
+    if (sum != a.budget) plan_bad = 1;
+    Fj = plan_bad ? 0 : sm.s_F[j];
+  }
+  if (plan_bad) flags |= SSD_ROW_BAD_PLAN;
+  const bool want_topf = has_plan && Fj > 0;
+  const bool fast_ok = want_topf && Fj <= kMaxGroups;
   SlicePart* part = a.parts + u * S + slice;
   if (warp == 0) {
     float m1 = -INFINITY, s1 = 0.f, m2 = -INFINITY, s2 = 0.f;
@@ -783,7 +815,7 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) ssd_stats_kernel(const _
         const int v = e0 + g1 * VE + i;
         if (x[i] >= tau && v < e1) {
           const int pos = atomicAdd(&sm.n_raw, 1);
-          if (pos < kCandCap) sm.raw[pos] = Cand{x[i], v};
+          if (pos < kCandCap) raw[pos] = Cand{x[i], v};
         }
       }
       if (vm2 >= tau && g2 >= 0) {
@@ -793,7 +825,7 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) ssd_stats_kernel(const _
           const int v = e0 + g2 * VE + i;
           if (x[i] >= tau && v < e1) {
             const int pos = atomicAdd(&sm.n_raw, 1);
-            if (pos < kCandCap) sm.raw[pos] = Cand{x[i], v};
+            if (pos < kCandCap) raw[pos] = Cand{x[i], v};
           }
         }
       }
@@ -810,7 +842,7 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) ssd_stats_kernel(const _
             const int v = e0 + g * VE + i;
             if (x[i] >= tau && v < e1) {
               const int pos = atomicAdd(&sm.n_raw, 1);
-              if (pos < kCandCap) sm.raw[pos] = Cand{x[i], v};
+              if (pos < kCandCap) raw[pos] = Cand{x[i], v};
             }
           }
         }
@@ -823,10 +855,10 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) ssd_stats_kernel(const _
     const int nr = min(sm.n_raw, kCandCap);
     const int keepn = min(min(nr, Fj), kCandSlice);
     for (int i = tid; i < nr; i += kThreads) {
-      const Cand ci = sm.raw[i];
+      const Cand ci = raw[i];
       const unsigned long long key = rank_key(ci.x, ci.idx);
       int r = 0;
-      for (int k2 = 0; k2 < nr; ++k2) r += rank_key(sm.raw[k2].x, sm.raw[k2].idx) > key;
+      for (int k2 = 0; k2 < nr; ++k2) r += rank_key(raw[k2].x, raw[k2].idx) > key;
       if (r < keepn) part->cand[r] = ci;
     }
     if (tid == 0) part->n_cand = sm.n_raw;
@@ -841,6 +873,17 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) ssd_stats_kernel(const _
 
   // =============== the unit's finalizer: the last slice to arrive ===================
   const SlicePart* parts = a.parts + u * S;
+  // Every slice's published candidates, loaded at once with the statistics
+  // (slot c * cap + r holds candidate r of slice c; entries past a slice's
+  // count are ignored).
+  const int cap = min(Fj, kCandSlice);
+  const bool one_round = fast_ok && S * cap <= kGatherCap;
+  if (one_round && warp != 0) {
+    for (int i = tid - 32; i < S * cap; i += kThreads - 32) {
+      const Cand* src = &parts[i / cap].cand[i % cap];
+      gbuf[i] = Cand{__ldcg(&src->x), __ldcg(&src->idx)};
+    }
+  }
   if (warp == 0) {
     // Butterfly over the slices (lanes >= S hold neutral values): bit-identical
     // results whichever CTA finalizes.
@@ -872,7 +915,10 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) ssd_stats_kernel(const _
     const int total = __shfl_sync(0xFFFFFFFFu, incl, 31);
     const unsigned over = __ballot_sync(0xFFFFFFFFu, nc > kCandCap || (nc > kCandSlice && Fj > kCandSlice));
     const unsigned anyto = __ballot_sync(0xFFFFFFFFu, to != 0);
-    if (lane < S) sm.cand_off[lane] = incl - cnt;
+    if (lane < S) {
+      sm.cand_off[lane] = incl - cnt;
+      sm.cnt[lane] = cnt;
+    }
     if (lane == 0) {
       sm.MP = mp; sm.SP = sp; sm.MQ = mq; sm.SQ = sq; sm.argP = ap; sm.argQ = aq;
       sm.cand_off[S] = total;
@@ -887,35 +933,28 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) ssd_stats_kernel(const _
   if (hasP && !(MP > -INFINITY && MP < INFINITY)) flags |= SSD_ROW_NONFINITE;
   if (hasQ && !(MQ > -INFINITY && MQ < INFINITY)) flags |= SSD_ROW_NONFINITE;
   const bool valid = (flags & SSD_ROW_INVALID) == 0;
-  const bool slow = want_topf && valid && (!fast_ok || sm.slow != 0);
-  Cand* sel = sm.buf + kGatherCap;
+  const bool slow = want_topf && valid && (!one_round || sm.slow != 0);
+  Cand* sel = gbuf + kGatherCap;
   const float nmP = -MP * cT, nmQ = -MQ * cT;
 
   // ---- exact top-F: global ranks by binary search in the sorted slice lists --------
   if (want_topf && valid && !slow) {
-    const int N = sm.n_total;
-    for (int i = tid; i < N; i += kThreads) {
-      int c = 0;
-      while (c + 1 < S && sm.cand_off[c + 1] <= i) ++c;
-      const Cand* src = &parts[c].cand[i - sm.cand_off[c]];
-      sm.buf[i] = Cand{__ldcg(&src->x), __ldcg(&src->idx)};
-    }
-    __syncthreads();
-    for (int i = tid; i < N; i += kThreads) {
-      int c = 0;
-      while (c + 1 < S && sm.cand_off[c + 1] <= i) ++c;
-      const Cand ci = sm.buf[i];
+    for (int i = tid; i < S * cap; i += kThreads) {
+      const int c = i / cap, r0 = i - c * cap;
+      if (r0 >= sm.cnt[c]) continue;
+      const Cand ci = gbuf[i];
       const unsigned long long key = rank_key(ci.x, ci.idx);
-      int r = i - sm.cand_off[c];  // entries ahead of it in its own list
+      int r = r0;  // entries ahead of it in its own list
       for (int c2 = 0; c2 < S; ++c2) {
         if (c2 == c) continue;
-        int lo = sm.cand_off[c2], hi = sm.cand_off[c2 + 1];  // count keys > key (descending list)
+        const int base = c2 * cap;
+        int lo = base, hi = base + sm.cnt[c2];  // count keys > key (descending list)
         while (lo < hi) {
           const int mid = (lo + hi) >> 1;
-          if (rank_key(sm.buf[mid].x, sm.buf[mid].idx) > key) lo = mid + 1;
+          if (rank_key(gbuf[mid].x, gbuf[mid].idx) > key) lo = mid + 1;
           else hi = mid;
         }
-        r += lo - sm.cand_off[c2];
+        r += lo - base;
       }
       if (r < Fj) sel[r] = ci;
     }
@@ -1018,11 +1057,14 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) ssd_stats_kernel(const _
         am = fminf(am, __ldcg(&us[k].amargin));
         if (__ldcg(&us[k].rejected)) { kstar = k; break; }
       }
+      const UnitState* uk = us + kstar;
       RowState rs;
       rs.kstar = kstar;
       rs.flags = fl;
       rs.amargin = am;
-      rs.pad = 0;
+      rs.Fj = __ldcg(&uk->Fj);
+      rs.MP = __ldcg(&uk->MP); rs.SP = __ldcg(&uk->SP); rs.MQ = __ldcg(&uk->MQ); rs.SQ = __ldcg(&uk->SQ);
+      rs.Z = __ldcg(&uk->Z); rs.bx = __ldcg(&uk->bx); rs.bi = __ldcg(&uk->bi); rs.argP = __ldcg(&uk->argP);
       a.rstate[b] = rs;
     } else {
       const bool pbad = (fl & SSD_ROW_BAD_PLAN) != 0;
@@ -1033,7 +1075,12 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) ssd_stats_kernel(const _
         a.offsets[static_cast<long long>(b) * (K + 2) + k + 1] = off;
       }
       if (!a.draws) a.status[b] = fl;
-      else a.rstate[b] = RowState{0, fl, INFINITY, 0};
+      else {
+        RowState rs = {};
+        rs.flags = fl;
+        rs.amargin = INFINITY;
+        a.rstate[b] = rs;
+      }
     }
     a.row_arrive[b] = 0;
   }
@@ -1094,7 +1141,7 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) ssd_draw_kernel(const __
   __shared__ __align__(16) Smem2 sm;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int S = a.n_slices;
+  const int S = a.d_slices;
   const int du = blockIdx.x / S, slice = blockIdx.x % S;
   const int K = a.K, V = a.V;
   const bool verify = a.mode == kModeVerify;
@@ -1102,6 +1149,7 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) ssd_draw_kernel(const __
   // ---- which unit this row (or draft position) draws from ----------------------------
   int b, j, rowflags = 0, draw;
   float amargin = INFINITY;
+  UnitState st;
   if (verify) {
     b = du;
     const RowState rs = a.rstate[b];
@@ -1109,13 +1157,16 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) ssd_draw_kernel(const __
     rowflags = rs.flags;
     amargin = rs.amargin;
     draw = j < K ? kDrawResidual : kDrawP;
+    st.MP = rs.MP; st.SP = rs.SP; st.MQ = rs.MQ; st.SQ = rs.SQ;
+    st.Z = rs.Z; st.bx = rs.bx; st.bi = rs.bi; st.argP = rs.argP; st.argQ = 0;
+    st.Fj = rs.Fj; st.flags = rowflags;
   } else {
     b = du / K;
     j = du % K;
     draw = kDrawQ;
+    st = a.ustate[static_cast<long long>(b) * (K + 1) + j];
   }
   const long long u = static_cast<long long>(b) * (K + 1) + j;
-  const UnitState st = a.ustate[u];
   const bool row_invalid = verify ? (rowflags & SSD_ROW_INVALID) != 0 : (st.flags & SSD_ROW_INVALID) != 0;
   const bool streams = !kGreedy && !row_invalid;
   if (!streams && slice != 0) return;
@@ -1124,8 +1175,8 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) ssd_draw_kernel(const __
   long long rbP, rbQ;
   unit_rows<TIn>(a, b, j, baseP, rbP, baseQ, rbQ);
   if (draw == kDrawP) baseQ = nullptr;  // the full-acceptance draw reads p_K only
-  const int e0 = slice * a.chunk;
-  const int e1 = min(V, e0 + a.chunk);
+  const int e0 = slice * a.d_chunk;
+  const int e1 = min(V, e0 + a.d_chunk);
   const int n = max(0, e1 - e0);
   const int nvec = (n + VE - 1) / VE;
   const int nch = (nvec + kChunkVecs - 1) / kChunkVecs;
@@ -1238,8 +1289,8 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) ssd_draw_kernel(const __
       const int s_star = sm.cstar;
       const bool use_p = sm.use_p != 0;
       const DrawPart* dp = &dparts[s_star];
-      const int e0s = s_star * a.chunk;
-      const int e1s = min(V, e0s + a.chunk);
+      const int e0s = s_star * a.d_chunk;
+      const int e1s = min(V, e0s + a.d_chunk);
       const int nvs = (max(0, e1s - e0s) + VE - 1) / VE;
       const int nchs = (nvs + kChunkVecs - 1) / kChunkVecs;
       const float tl = sm.tl;
