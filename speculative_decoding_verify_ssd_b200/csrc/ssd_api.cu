@@ -168,7 +168,8 @@ static cudaError_t prepare_kernel(const void* fn) {
 // Workspace: slice partials, unit states, draw partials, row states, then the
 // counters (zero between calls) and the error word.
 struct WsLayout {
-  size_t parts, ustate, dparts, rstate, arrive1, row_arrive, draw_arrive, row_arrive2, error, total;
+  size_t parts, ustate, dparts, rstate, arrive1, row_arrive, draw_arrive, row_arrive2, rflag, epoch, k2_done, error,
+      total;
   int n_slices;
 };
 
@@ -202,6 +203,9 @@ static WsLayout ws_layout(int B, int K, int V, int dtype) {
   w.row_arrive = off;  off += nb * sizeof(int32_t);
   w.draw_arrive = off; off += nb * static_cast<size_t>(K) * sizeof(int32_t);
   w.row_arrive2 = off; off += nb * sizeof(int32_t);
+  w.rflag = off;       off += nb * static_cast<size_t>(K) * sizeof(int32_t);
+  w.epoch = off;       off += sizeof(uint32_t);
+  w.k2_done = off;     off += sizeof(int32_t);
   w.error = off;       off += sizeof(int32_t);
   w.total = up256(off);
   return w;
@@ -217,6 +221,9 @@ static void bind_workspace(Args& a, void* ws, const WsLayout& w) {
   a.row_arrive = reinterpret_cast<int32_t*>(base + w.row_arrive);
   a.draw_arrive = reinterpret_cast<int32_t*>(base + w.draw_arrive);
   a.row_arrive2 = reinterpret_cast<int32_t*>(base + w.row_arrive2);
+  a.rflag = reinterpret_cast<int32_t*>(base + w.rflag);
+  a.epoch = reinterpret_cast<uint32_t*>(base + w.epoch);
+  a.k2_done = reinterpret_cast<int32_t*>(base + w.k2_done);
   a.error = reinterpret_cast<int32_t*>(base + w.error);
 }
 
@@ -230,9 +237,19 @@ static ssd_status launch_t(const Args& a, long long units, long long draw_units,
       <<<static_cast<unsigned>(units * a.n_slices), kThreads, smem, stream>>>(a);
   if (cudaGetLastError() != cudaSuccess) return SSD_ERR_CUDA;
   if (draw_units > 0) {
-    ssd_draw_kernel<TIn, kAligned, kGreedy>
-        <<<static_cast<unsigned>(draw_units * a.d_slices), kThreads, smem, stream>>>(a);
-    if (cudaGetLastError() != cudaSuccess) return SSD_ERR_CUDA;
+    // Programmatic dependent launch: the draw kernel may start while the
+    // stats kernel finishes; each of its CTAs waits for its own row decision.
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(draw_units * a.d_slices));
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, ssd_draw_kernel<TIn, kAligned, kGreedy>, a) != cudaSuccess) return SSD_ERR_CUDA;
   }
   return SSD_OK;
 }

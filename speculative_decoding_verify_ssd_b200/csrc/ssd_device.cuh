@@ -69,6 +69,37 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
   return false;
 }
 
+// Acquire load / release store of a flag in global memory, GPU scope.
+__device__ __forceinline__ int32_t ld_acquire_gpu(const int32_t* p) {
+  int32_t v;
+  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ void st_release_gpu(int32_t* p, int32_t v) {
+  asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+// Nanoseconds of the GPU's global timer.
+__device__ __forceinline__ unsigned long long global_ns() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+// Bounded wait for a flag written by another CTA (or grid): true once
+// *flag == want; false after `limit_ns` of waiting (or as many polls).
+__device__ __forceinline__ bool wait_flag(const int32_t* flag, int32_t want, unsigned long long limit_ns) {
+  const unsigned long long t0 = global_ns();
+  uint32_t sleep_ns = 64;
+  for (uint32_t i = 0; i < 50000000u; ++i) {
+    if (ld_acquire_gpu(flag) == want) return true;
+    if (global_ns() - t0 > limit_ns) return false;
+    __nanosleep(sleep_ns);
+    if (sleep_ns < 1024) sleep_ns <<= 1;
+  }
+  return false;
+}
+
 // 1-D bulk copy global -> this CTA's shared memory (no multicast).  Both
 // addresses 16-byte aligned, bytes a multiple of 16.
 __device__ __forceinline__ void bulk_copy_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {

@@ -55,6 +55,7 @@ constexpr int kSelCap = 512;           // >= SSD_MAX_BUDGET
 constexpr int kMaxGroups = kThreads;   // thread maxima per CTA
 constexpr uint32_t kMaxPolls = 4000000u;  // x ~0.5 us sleep: about 2 s
 constexpr float kNearTie = 1e-5f;
+constexpr unsigned long long kDepWaitNs = 1000000000ull;  // a draw's wait for its row decision
 constexpr int kFlagTimeout = SSD_ROW_DEVICE_TIMEOUT;
 constexpr size_t kRingBytes = static_cast<size_t>(kStages) * 2 * kChunkVecs * 16;
 
@@ -148,6 +149,9 @@ struct Args {
   int32_t* row_arrive;
   int32_t* draw_arrive;
   int32_t* row_arrive2;
+  int32_t* rflag;          // per draw unit: epoch + 1 once the row decision is written
+  uint32_t* epoch;         // calls completed on this workspace (kernel 2 advances it)
+  int32_t* k2_done;        // kernel 2 CTAs past their wait
   int32_t* error;
 };
 
@@ -599,7 +603,12 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) ssd_stats_kernel(const _
   const int S = a.n_slices;
   const int order = blockIdx.x / S, slice = blockIdx.x % S;
   const int upr = a.units_per_row;
-  const int b = order % a.B, j = (upr - 1) - order / a.B;  // decreasing position order
+  // rows in order, so that rows are decided (and their draws may start) one
+  // after another; within a row, positions from the last
+  const int b = order / upr, j = (upr - 1) - order % upr;
+  // kernel 2 may be scheduled once every CTA of this grid has started; it
+  // waits for each row's decision on its own
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int K = a.K, V = a.V;
   const bool verify = a.mode == kModeVerify;
   const long long u = static_cast<long long>(b) * (K + 1) + j;
@@ -1066,6 +1075,8 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) ssd_stats_kernel(const _
       rs.MP = __ldcg(&uk->MP); rs.SP = __ldcg(&uk->SP); rs.MQ = __ldcg(&uk->MQ); rs.SQ = __ldcg(&uk->SQ);
       rs.Z = __ldcg(&uk->Z); rs.bx = __ldcg(&uk->bx); rs.bi = __ldcg(&uk->bi); rs.argP = __ldcg(&uk->argP);
       a.rstate[b] = rs;
+      __threadfence();
+      st_release_gpu(a.rflag + b, static_cast<int32_t>(*reinterpret_cast<volatile uint32_t*>(a.epoch) + 1u));
     } else {
       const bool pbad = (fl & SSD_ROW_BAD_PLAN) != 0;
       int off = 0;
@@ -1080,6 +1091,9 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) ssd_stats_kernel(const _
         rs.flags = fl;
         rs.amargin = INFINITY;
         a.rstate[b] = rs;
+        __threadfence();
+        const int32_t want = static_cast<int32_t>(*reinterpret_cast<volatile uint32_t*>(a.epoch) + 1u);
+        for (int k = 0; k < K; ++k) st_release_gpu(a.rflag + static_cast<long long>(b) * K + k, want);
       }
     }
     a.row_arrive[b] = 0;
@@ -1089,6 +1103,7 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) ssd_stats_kernel(const _
 // Shared memory of kernel 2.
 struct Smem2 {
   uint64_t full[kStages];
+  int32_t dep_ok;
   float rs[kMaxChunks][kWarps];
   float ps[kMaxChunks][kWarps];
   int32_t s_F[SSD_MAX_K + 1];
@@ -1146,13 +1161,36 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) ssd_draw_kernel(const __
   const int K = a.K, V = a.V;
   const bool verify = a.mode == kModeVerify;
 
+  // ---- the row decision this CTA needs (kernel 1 may still be running) -------------
+  if (tid == 0) {
+    const uint32_t epoch = *reinterpret_cast<volatile const uint32_t*>(a.epoch);
+    sm.dep_ok = wait_flag(a.rflag + du, static_cast<int32_t>(epoch + 1u), kDepWaitNs) ? 1 : 0;
+    if (atomicAdd(a.k2_done, 1) == static_cast<int>(gridDim.x) - 1) {  // every CTA has read the epoch
+      *a.k2_done = 0;
+      __threadfence();
+      atomicAdd(a.epoch, 1u);
+    }
+  }
+  __syncthreads();
+  const bool dep_ok = sm.dep_ok != 0;
+
   // ---- which unit this row (or draft position) draws from ----------------------------
   int b, j, rowflags = 0, draw;
   float amargin = INFINITY;
   UnitState st;
   if (verify) {
     b = du;
-    const RowState rs = a.rstate[b];
+    RowState rs;
+    rs.kstar = __ldcg(&a.rstate[b].kstar); rs.flags = __ldcg(&a.rstate[b].flags);
+    rs.amargin = __ldcg(&a.rstate[b].amargin); rs.Fj = __ldcg(&a.rstate[b].Fj);
+    rs.MP = __ldcg(&a.rstate[b].MP); rs.SP = __ldcg(&a.rstate[b].SP);
+    rs.MQ = __ldcg(&a.rstate[b].MQ); rs.SQ = __ldcg(&a.rstate[b].SQ);
+    rs.Z = __ldcg(&a.rstate[b].Z); rs.bx = __ldcg(&a.rstate[b].bx);
+    rs.bi = __ldcg(&a.rstate[b].bi); rs.argP = __ldcg(&a.rstate[b].argP);
+    if (!dep_ok || rs.kstar < 0 || rs.kstar > K) {  // the decision never came: a timed-out row
+      rs.kstar = K;
+      rs.flags = kFlagTimeout;
+    }
     j = rs.kstar;
     rowflags = rs.flags;
     amargin = rs.amargin;
@@ -1164,7 +1202,11 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) ssd_draw_kernel(const __
     b = du / K;
     j = du % K;
     draw = kDrawQ;
-    st = a.ustate[static_cast<long long>(b) * (K + 1) + j];
+    const UnitState* us = a.ustate + static_cast<long long>(b) * (K + 1) + j;
+    st.MQ = __ldcg(&us->MQ); st.SQ = __ldcg(&us->SQ); st.Z = __ldcg(&us->Z); st.bx = __ldcg(&us->bx);
+    st.bi = __ldcg(&us->bi); st.argQ = __ldcg(&us->argQ); st.Fj = __ldcg(&us->Fj);
+    st.flags = __ldcg(&us->flags) | (dep_ok ? 0 : kFlagTimeout);
+    st.MP = 0.f; st.SP = 1.f; st.argP = 0;
   }
   const long long u = static_cast<long long>(b) * (K + 1) + j;
   const bool row_invalid = verify ? (rowflags & SSD_ROW_INVALID) != 0 : (st.flags & SSD_ROW_INVALID) != 0;
@@ -1391,7 +1433,7 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) ssd_draw_kernel(const __
       sm.is_last_row = atomicAdd(a.row_arrive2 + b, 1) == K - 1;
       if (sm.is_last_row) {
         __threadfence();
-        int fl = a.rstate[b].flags;
+        int fl = __ldcg(&a.rstate[b].flags);
         for (int k = 0; k < K; ++k) {
           const UnitState* uk = a.ustate + static_cast<long long>(b) * (K + 1) + k;
           fl |= __ldcg(&uk->flags);
