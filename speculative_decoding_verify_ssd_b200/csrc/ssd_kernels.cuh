@@ -639,8 +639,8 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) ssd_stats_kernel(const _
   if constexpr (kAligned) ring.start(tid);
 
   const bool has_plan = a.F != nullptr || a.alpha != nullptr;
-  // The plan's inputs are loaded now; warp 0 forms the plan after the stream
-  // (only the epilogue needs it).
+  // Warp 0 forms the plan now, while the first chunks are in flight (only the
+  // epilogue reads it; the stream's first barrier publishes it).
   int fplan[2] = {0, 0};
   float alpha_in = 0.f;
   if (warp == 0 && has_plan) {
@@ -652,6 +652,12 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) ssd_stats_kernel(const _
       }
     } else if (a.fanout_mode != SSD_FANOUT_UNIFORM && lane == 0) {
       alpha_in = __ldg(a.alpha + b);
+    }
+    if (!a.F) fanout_warp(__shfl_sync(0xFFFFFFFFu, alpha_in, 0), K, a.budget, a.fanout_mode, lane, fplan);
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int k = lane + 32 * h;
+      if (k <= K) sm.s_F[k] = fplan[h];
     }
   }
   int flags = 0, d = -1;
@@ -720,14 +726,6 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) ssd_stats_kernel(const _
   }
   if constexpr (kGreedy) {
     if (nan_seen) { mP = __int_as_float(0x7FC00000); mQ = mP; }
-  }
-  if (warp == 0 && has_plan) {
-    if (!a.F) fanout_warp(__shfl_sync(0xFFFFFFFFu, alpha_in, 0), K, a.budget, a.fanout_mode, lane, fplan);
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const int k = lane + 32 * h;
-      if (k <= K) sm.s_F[k] = fplan[h];
-    }
   }
   sm.gmax[tid] = vm1;
   if (tid == 0) sm.n_raw = 0;
@@ -1165,6 +1163,7 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) ssd_draw_kernel(const __
   if (tid == 0) {
     const uint32_t epoch = *reinterpret_cast<volatile const uint32_t*>(a.epoch);
     sm.dep_ok = wait_flag(a.rflag + du, static_cast<int32_t>(epoch + 1u), kDepWaitNs) ? 1 : 0;
+    if (!sm.dep_ok) atomicExch(a.error, 1);
     if (atomicAdd(a.k2_done, 1) == static_cast<int>(gridDim.x) - 1) {  // every CTA has read the epoch
       *a.k2_done = 0;
       __threadfence();
