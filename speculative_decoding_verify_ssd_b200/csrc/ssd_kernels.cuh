@@ -21,12 +21,15 @@
 //   top-F by (logit desc, token id asc), forms Q_S and the Saguaro normaliser
 //   Z = 1 - (1 - C) Q_S ([ZH] challenge 2; [NL] 3B), and runs the lossless
 //   accept test a_j = min(1, p_j(d_j) / q'_j(d_j)); the last unit of a row
-//   fixes k*, the first rejected position.  Units are issued in decreasing
-//   position order, so the rows most often needed next are still in L2.
+//   fixes k*, the first rejected position, and raises the row's flag.  Rows
+//   are taken in order, so they are decided one after another.
 //
 // Kernel 2 (draw): one CTA per (row, slice) of the single unit each row
 //   draws from: the residual r = max(0, p_k* - q'_k*) (or p_K after full
-//   acceptance, or q' for a draft draw).  Each CTA sums its slice of r per
+//   acceptance, or q' for a draft draw).  It is a programmatic dependent of
+//   kernel 1 (scheduled once every kernel-1 CTA has started) and each CTA
+//   waits only for its own row's flag, so the draws of early rows run while
+//   kernel 1 finishes.  Each CTA sums its slice of r per
 //   (ring chunk, warp); the last CTA of the row finds where the cumulative
 //   mass crosses u * R in token order (slice, chunk, warp, then one re-read
 //   vector per lane), draws the bonus token, and finishes the row: outputs,
