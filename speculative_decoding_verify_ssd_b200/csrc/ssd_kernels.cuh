@@ -49,7 +49,10 @@ constexpr int kWarps = kThreads / 32;
 constexpr int kMinBlocks = 4;          // CTAs per SM the register budget is set for
 constexpr int kMaxSlices = 16;         // slices per logit row
 constexpr int kStages = 6;             // depth of the bulk-copy ring
-constexpr int kChunkVecs = kThreads;   // 16-byte vectors per row per ring stage
+constexpr int kChunkVecs = kThreads;   // 16-byte vectors per row per ring stage (draw kernel)
+constexpr int kStatsVPT = 2;           // stats kernel: vectors per thread per row per stage
+constexpr int kStatsChunkVecs = kChunkVecs * kStatsVPT;
+constexpr int kStatsStages = kStages * kChunkVecs / kStatsChunkVecs;  // same ring bytes
 constexpr int kMaxChunks = 16;         // ring chunks per slice
 constexpr int kCandCap = 256;          // local top-F candidates found by a CTA
 constexpr int kCandSlice = 128;        // candidates a slice publishes
@@ -420,10 +423,10 @@ __device__ __forceinline__ void fanout_row(float alpha_f, int K, int budget, int
 
 
 // Ring of bulk copies that streams one slice of up to two rows of a unit
-// through shared memory, chunk by chunk (one 16-byte vector per thread per row
-// and chunk).  Thread 0 issues and polls; the other threads sleep in the CTA
-// barrier and then take one acquiring look at the stage's phase.
-template <typename TIn>
+// through shared memory, chunk by chunk (CV 16-byte vectors per row per
+// chunk, ST stages).  Thread 0 issues and polls; the other threads sleep in the
+// CTA barrier and then take one acquiring look at the stage's phase.
+template <typename TIn, int CV = kChunkVecs, int ST = kStages>
 struct Ring {
   unsigned char* buf;
   uint64_t* full;
@@ -432,13 +435,13 @@ struct Ring {
   int nrows, e0, nvec, nch, n_issued;
 
   __device__ __forceinline__ unsigned char* stage(int slot, int r) const {
-    return buf + (static_cast<size_t>(slot) * 2 + r) * (kChunkVecs * 16);
+    return buf + (static_cast<size_t>(slot) * 2 + r) * (CV * 16);
   }
   __device__ __forceinline__ void issue(int c) {
     constexpr int VE = 16 / sizeof(TIn);
-    const int slot = c % kStages;
-    const int v0 = c * kChunkVecs;
-    const int nv = min(kChunkVecs, nvec - v0);
+    const int slot = c % ST;
+    const int v0 = c * CV;
+    const int nv = min(CV, nvec - v0);
     mbar_arrive_expect_tx(&full[slot], static_cast<uint32_t>(nv) * 16u * static_cast<uint32_t>(nrows));
     bulk_copy_g2s(stage(slot, 0), row0 + e0 + v0 * VE, static_cast<uint32_t>(nv) * 16u, &full[slot]);
     if (nrows > 1) bulk_copy_g2s(stage(slot, 1), row1 + e0 + v0 * VE, static_cast<uint32_t>(nv) * 16u, &full[slot]);
@@ -447,29 +450,29 @@ struct Ring {
   __device__ __forceinline__ void start(int tid) {
     n_issued = 0;
     if (tid == 0) {
-      for (int s = 0; s < kStages; ++s) mbar_init(&full[s], 1);
+      for (int s = 0; s < ST; ++s) mbar_init(&full[s], 1);
       mbar_init_fence();
     }
     __syncthreads();
     if (tid == 0)
-      for (int c = 0; c < min(kStages, nch); ++c) issue(c);
+      for (int c = 0; c < min(ST, nch); ++c) issue(c);
   }
   // Chunk c is ready for every thread; the barrier also marks chunk c - 1
   // consumed, so its stage is refilled.
   __device__ __forceinline__ void acquire(int c, int tid, int& tmo) {
-    if (tid == 0 && !mbar_wait_bounded(&full[c % kStages], (c / kStages) & 1, kMaxPolls)) tmo = 1;
+    if (tid == 0 && !mbar_wait_bounded(&full[c % ST], (c / ST) & 1, kMaxPolls)) tmo = 1;
     __syncthreads();
-    if (tid == 0 && c > 0 && c - 1 + kStages < nch) issue(c - 1 + kStages);
-    if (tid != 0 && !mbar_try_wait(&full[c % kStages], (c / kStages) & 1, 0u)) tmo = 1;
+    if (tid == 0 && c > 0 && c - 1 + ST < nch) issue(c - 1 + ST);
+    if (tid != 0 && !mbar_try_wait(&full[c % ST], (c / ST) & 1, 0u)) tmo = 1;
   }
   __device__ __forceinline__ uint4 vec(int c, int r, int tid) const {
-    return *reinterpret_cast<const uint4*>(stage(c % kStages, r) + tid * 16);
+    return *reinterpret_cast<const uint4*>(stage(c % ST, r) + tid * 16);
   }
   // Never leave a copy in flight (only a timed-out wait can leave one).
   __device__ __forceinline__ void drain(int tid, int tmo) {
     if (tmo && tid == 0)
-      for (int c = max(0, n_issued - kStages); c < n_issued; ++c)
-        mbar_wait_bounded(&full[c % kStages], (c / kStages) & 1, kMaxPolls);
+      for (int c = max(0, n_issued - ST); c < n_issued; ++c)
+        mbar_wait_bounded(&full[c % ST], (c / ST) & 1, kMaxPolls);
   }
 };
 
@@ -628,8 +631,8 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) ssd_stats_kernel(const _
   const int e1 = min(V, e0 + a.chunk);
   const int n = max(0, e1 - e0);
   const int nvec = (n + VE - 1) / VE;
-  const int nch = (nvec + kChunkVecs - 1) / kChunkVecs;
-  Ring<TIn> ring;
+  const int nch = (nvec + kStatsChunkVecs - 1) / kStatsChunkVecs;
+  Ring<TIn, kStatsChunkVecs, kStatsStages> ring;
   ring.buf = ring_buf;
   ring.full = sm.full;
   ring.row0 = hasP ? baseP + rbP : baseQ + rbQ;
@@ -686,7 +689,10 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) ssd_stats_kernel(const _
   uint4 keep1 = make_uint4(0u, 0u, 0u, 0u), keep2 = keep1;  // the source vectors holding vm1, vm2
   for (int c = 0; c < nch; ++c) {
     if constexpr (kAligned) ring.acquire(c, tid, tmo);
-    const int g = c * kChunkVecs + tid;
+#pragma unroll
+    for (int v = 0; v < kStatsVPT; ++v) {
+    const int t = v * kChunkVecs + tid;  // the thread's vector within the chunk
+    const int g = c * kStatsChunkVecs + t;
     if (g < nvec) {
       const int vbase = e0 + g * VE;
       float vsrc;
@@ -694,9 +700,9 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) ssd_stats_kernel(const _
       if constexpr (kAligned && sizeof(TIn) == 2) {
         float vp = -INFINITY;
         uint4 wq = make_uint4(0u, 0u, 0u, 0u), wp = wq;
-        if (hasP) { wp = ring.vec(c, slotP, tid); vp = consume_bf16<kGreedy>(wp, vbase, cT, mP, sP, nmP1, argP, nan_seen); }
+        if (hasP) { wp = ring.vec(c, slotP, t); vp = consume_bf16<kGreedy>(wp, vbase, cT, mP, sP, nmP1, argP, nan_seen); }
         float vq = -INFINITY;
-        if (hasQ) { wq = ring.vec(c, slotQ, tid); vq = consume_bf16<kGreedy>(wq, vbase, cT, mQ, sQ, nmQ1, argQ, nan_seen); }
+        if (hasQ) { wq = ring.vec(c, slotQ, t); vq = consume_bf16<kGreedy>(wq, vbase, cT, mQ, sQ, nmQ1, argQ, nan_seen); }
         vsrc = srcQ ? vq : vp;
         wsrc = srcQ ? wq : wp;
       } else {
@@ -704,12 +710,12 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) ssd_stats_kernel(const _
         float vp = -INFINITY, vq = -INFINITY;
         uint4 wp = make_uint4(0u, 0u, 0u, 0u), wq = wp;
         if (hasP) {
-          if constexpr (kAligned) { wp = ring.vec(c, slotP, tid); Elem<TIn>::unpack(wp, x); }
+          if constexpr (kAligned) { wp = ring.vec(c, slotP, t); Elem<TIn>::unpack(wp, x); }
           else load_group<TIn, false>(baseP, rbP, vbase, e1, x);
           vp = consume_f<VE, kGreedy>(x, vbase, cT, mP, sP, nmP1, argP, nan_seen);
         }
         if (hasQ) {
-          if constexpr (kAligned) { wq = ring.vec(c, slotQ, tid); Elem<TIn>::unpack(wq, x); }
+          if constexpr (kAligned) { wq = ring.vec(c, slotQ, t); Elem<TIn>::unpack(wq, x); }
           else load_group<TIn, false>(baseQ, rbQ, vbase, e1, x);
           vq = consume_f<VE, kGreedy>(x, vbase, cT, mQ, sQ, nmQ1, argQ, nan_seen);
         }
@@ -725,6 +731,7 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) ssd_stats_kernel(const _
           vm3 = vsrc;
         }
       }
+    }
     }
   }
   if constexpr (kGreedy) {
@@ -842,9 +849,8 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) ssd_stats_kernel(const _
     } else {
       const TIn* bs = srcQ ? baseQ : baseP;
       const long long rs = srcQ ? rbQ : rbP;
-      for (int c = 0; c < nch; ++c) {
-        const int g = c * kChunkVecs + tid;
-        if (g < nvec) {
+      for (int g = tid; g < nvec; g += kThreads) {
+        {
           float x[VE];
           load_group<TIn, kAligned>(bs, rs, e0 + g * VE, e1, x);
 #pragma unroll
