@@ -55,16 +55,24 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity, ui
   return done != 0;
 }
 
-// Bounded wait: polls, and between unsuccessful polls puts the warp to sleep
-// (exponential backoff up to ~0.5 us) so that a waiting warp does not take
-// issue slots from co-resident CTAs.  Gives up after `max_polls` polls and
-// returns false.
-__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, uint32_t max_polls) {
-  uint32_t sleep_ns = 32;
-  for (uint32_t i = 0; i < max_polls; ++i) {
-    if (mbar_try_wait(bar, parity, 0u)) return true;
-    __nanosleep(sleep_ns);
-    if (sleep_ns < 512) sleep_ns <<= 1;
+// Nanoseconds of the GPU's global timer.
+__device__ __forceinline__ unsigned long long global_ns() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+// Bounded wait for a phase of an mbarrier.  Each poll suspends the thread in
+// hardware until the phase completes (or `kSuspendHintNs` pass), so a waiting
+// warp issues almost no instructions and resumes as soon as the bytes land.
+// Returns false once `limit_ns` of global time has passed without completion.
+constexpr uint32_t kSuspendHintNs = 100000u;
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, unsigned long long limit_ns) {
+  if (mbar_try_wait(bar, parity, kSuspendHintNs)) return true;
+  const unsigned long long t0 = global_ns();
+  for (uint32_t i = 0; i < (1u << 30); ++i) {
+    if (mbar_try_wait(bar, parity, kSuspendHintNs)) return true;
+    if (global_ns() - t0 > limit_ns) return false;
   }
   return false;
 }
@@ -79,12 +87,17 @@ __device__ __forceinline__ void st_release_gpu(int32_t* p, int32_t v) {
   asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 
-// Nanoseconds of the GPU's global timer.
-__device__ __forceinline__ unsigned long long global_ns() {
-  unsigned long long t;
-  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-  return t;
+// One thread's arrival on a counter in global memory, GPU scope, acquire and
+// release at once.  Issued after a CTA barrier, the release publishes what the
+// whole CTA wrote before the barrier (the barrier orders those writes before
+// this thread's), and after the next barrier the acquire makes what the
+// earlier arrivals published visible to the whole CTA.  Returns the old value.
+__device__ __forceinline__ int32_t arrive_acq_rel_gpu(int32_t* p) {
+  int32_t old;
+  asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], 1;" : "=r"(old) : "l"(p) : "memory");
+  return old;
 }
+
 
 // Bounded wait for a flag written by another CTA (or grid): true once
 // *flag == want; false after `limit_ns` of waiting (or as many polls).

@@ -59,7 +59,7 @@ constexpr int kCandSlice = 128;        // candidates a slice publishes
 constexpr int kGatherCap = 1024;       // candidates of a whole unit
 constexpr int kSelCap = 512;           // >= SSD_MAX_BUDGET
 constexpr int kMaxGroups = kThreads;   // thread maxima per CTA
-constexpr uint32_t kMaxPolls = 4000000u;  // x ~0.5 us sleep: about 2 s
+constexpr unsigned long long kRingWaitNs = 2000000000ull;  // a ring stage's bytes: 2 s at most
 constexpr float kNearTie = 1e-5f;
 constexpr unsigned long long kDepWaitNs = 1000000000ull;  // a draw's wait for its row decision
 constexpr int kFlagTimeout = SSD_ROW_DEVICE_TIMEOUT;
@@ -80,6 +80,7 @@ struct SlicePart {
   float mP, sP, mQ, sQ;           // running max and exp-sum of the slice
   int32_t argP, argQ;             // greedy: lowest id of the slice maximum
   int32_t n_cand, timeout;        // local candidates found; copy timeout
+  float xdP, xdQ;                 // logits of the drafted token (the slice that holds it)
   Cand cand[kCandSlice];          // sorted local candidates (at most min(n_cand, F))
 };
 
@@ -460,7 +461,7 @@ struct Ring {
   // Chunk c is ready for every thread; the barrier also marks chunk c - 1
   // consumed, so its stage is refilled.
   __device__ __forceinline__ void acquire(int c, int tid, int& tmo) {
-    if (tid == 0 && !mbar_wait_bounded(&full[c % ST], (c / ST) & 1, kMaxPolls)) tmo = 1;
+    if (tid == 0 && !mbar_wait_bounded(&full[c % ST], (c / ST) & 1, kRingWaitNs)) tmo = 1;
     __syncthreads();
     if (tid == 0 && c > 0 && c - 1 + ST < nch) issue(c - 1 + ST);
     if (tid != 0 && !mbar_try_wait(&full[c % ST], (c / ST) & 1, 0u)) tmo = 1;
@@ -472,7 +473,7 @@ struct Ring {
   __device__ __forceinline__ void drain(int tid, int tmo) {
     if (tmo && tid == 0)
       for (int c = max(0, n_issued - ST); c < n_issued; ++c)
-        mbar_wait_bounded(&full[c % ST], (c / ST) & 1, kMaxPolls);
+        mbar_wait_bounded(&full[c % ST], (c / ST) & 1, kRingWaitNs);
   }
 };
 
@@ -595,6 +596,8 @@ struct Smem1 {
   int32_t s_F[SSD_MAX_K + 1];
   float tau, MP, SP, MQ, SQ, QS, bx;
   int32_t bi, argP, argQ, n_total, slow, tmo, n_raw, is_last, is_last_row, pad;
+  int32_t Fj, seg_off, plan_bad;
+  float xdP, xdQ;
   int32_t cand_off[kMaxSlices + 1];
   int32_t cnt[kMaxSlices];
 };
@@ -660,10 +663,31 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) ssd_stats_kernel(const _
       alpha_in = __ldg(a.alpha + b);
     }
     if (!a.F) fanout_warp(__shfl_sync(0xFFFFFFFFu, alpha_in, 0), K, a.budget, a.fanout_mode, lane, fplan);
+    // the plan's checks (0 <= F <= V, sum = budget) and this unit's share
+    long long sum = 0;
+    int bad = 0, pre = 0, fj = 0;
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
       const int k = lane + 32 * h;
-      if (k <= K) sm.s_F[k] = fplan[h];
+      if (k <= K) {
+        const int f = fplan[h];
+        sm.s_F[k] = f;
+        bad |= (f < 0 || f > V) ? 1 : 0;
+        sum += f;
+        if (k < j) pre += f;
+        if (k == j) fj = f;
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xFFFFFFFFu, sum, o);
+    bad = __reduce_or_sync(0xFFFFFFFFu, bad);
+    pre = static_cast<int>(__reduce_add_sync(0xFFFFFFFFu, static_cast<unsigned>(pre)));
+    fj = static_cast<int>(__reduce_add_sync(0xFFFFFFFFu, static_cast<unsigned>(fj)));
+    if (lane == 0) {
+      const int pb = (bad || sum != a.budget) ? 1 : 0;
+      sm.plan_bad = pb;
+      sm.Fj = pb ? 0 : fj;
+      sm.seg_off = pre;
     }
   }
   int flags = 0, d = -1;
@@ -737,6 +761,13 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) ssd_stats_kernel(const _
   if constexpr (kGreedy) {
     if (nan_seen) { mP = __int_as_float(0x7FC00000); mQ = mP; }
   }
+  // The slice that holds the drafted token reads its two logits for the
+  // unit's accept test now (this CTA has just streamed them through L2).
+  float xdP = 0.f, xdQ = 0.f;
+  if (!kGreedy && has_d && tid == 0 && d >= e0 && d < e1) {
+    xdP = Elem<TIn>::at(baseP + rbP, d);
+    xdQ = Elem<TIn>::at(baseQ + rbQ, d);
+  }
   sm.gmax[tid] = vm1;
   if (tid == 0) sm.n_raw = 0;
 
@@ -756,10 +787,21 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) ssd_stats_kernel(const _
       sm.wint[warp][0] = argP; sm.wint[warp][1] = argQ;
     }
   } else {
+    // the warp's maxima first, then every lane rescales its sum once to them
+    float wmP = mP, wmQ = mQ;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
-      merge_ms(mP, sP, __shfl_xor_sync(0xFFFFFFFFu, mP, o), __shfl_xor_sync(0xFFFFFFFFu, sP, o), cT);
-      merge_ms(mQ, sQ, __shfl_xor_sync(0xFFFFFFFFu, mQ, o), __shfl_xor_sync(0xFFFFFFFFu, sQ, o), cT);
+      wmP = fmax_nan(wmP, __shfl_xor_sync(0xFFFFFFFFu, wmP, o));
+      wmQ = fmax_nan(wmQ, __shfl_xor_sync(0xFFFFFFFFu, wmQ, o));
+    }
+    sP = (mP == -INFINITY) ? 0.f : sP * ex2((mP - wmP) * cT);
+    sQ = (mQ == -INFINITY) ? 0.f : sQ * ex2((mQ - wmQ) * cT);
+    mP = wmP;
+    mQ = wmQ;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      sP += __shfl_xor_sync(0xFFFFFFFFu, sP, o);
+      sQ += __shfl_xor_sync(0xFFFFFFFFu, sQ, o);
     }
     if (lane == 0) {
       sm.wred[warp][0] = mP; sm.wred[warp][1] = sP;
@@ -769,15 +811,9 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) ssd_stats_kernel(const _
   tmo = __syncthreads_or(tmo);
   int Fj = 0, seg_off = 0, plan_bad = 0;
   if (has_plan) {
-    long long sum = 0;
-    for (int k = 0; k <= K; ++k) {
-      const int f = sm.s_F[k];
-      if (f < 0 || f > V) plan_bad = 1;
-      if (k < j) seg_off += f;
-      sum += f;
-    }
-    if (sum != a.budget) plan_bad = 1;
-    Fj = plan_bad ? 0 : sm.s_F[j];
+    plan_bad = sm.plan_bad;
+    Fj = sm.Fj;
+    seg_off = sm.seg_off;
   }
   if (plan_bad) flags |= SSD_ROW_BAD_PLAN;
   const bool want_topf = has_plan && Fj > 0;
@@ -805,6 +841,7 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) ssd_stats_kernel(const _
       part->mQ = m2; part->sQ = kGreedy ? 0.f : s2;
       part->argP = a1; part->argQ = a2;
       part->timeout = tmo;
+      part->xdP = xdP; part->xdQ = xdQ;
     }
   } else if (warp == 1) {
     // This slice's threshold: the F-th largest of its thread maxima bounds the
@@ -879,13 +916,11 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) ssd_stats_kernel(const _
     }
     if (tid == 0) part->n_cand = sm.n_raw;
   }
-  __threadfence();
   __syncthreads();
   if constexpr (kAligned) ring.drain(tid, tmo);
-  if (tid == 0) sm.is_last = atomicAdd(a.arrive1 + u, 1) == S - 1;
+  if (tid == 0) sm.is_last = arrive_acq_rel_gpu(a.arrive1 + u) == S - 1;
   __syncthreads();
   if (!sm.is_last) return;
-  __threadfence();
 
   // =============== the unit's finalizer: the last slice to arrive ===================
   const SlicePart* parts = a.parts + u * S;
@@ -911,6 +946,14 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) ssd_stats_kernel(const _
       ap = __ldcg(&parts[lane].argP); aq = __ldcg(&parts[lane].argQ);
       nc = __ldcg(&parts[lane].n_cand); to = __ldcg(&parts[lane].timeout);
     }
+    float xp = 0.f, xq = 0.f;
+    if (!kGreedy && has_d && lane < S) {
+      xp = __ldcg(&parts[lane].xdP);
+      xq = __ldcg(&parts[lane].xdQ);
+    }
+    const int cd = (has_d && d >= 0 && d < V) ? d / a.chunk : 0;  // the slice holding d
+    xp = __shfl_sync(0xFFFFFFFFu, xp, cd);
+    xq = __shfl_sync(0xFFFFFFFFu, xq, cd);
     const int cnt = min(min(nc, Fj), kCandSlice);
 #pragma unroll
     for (int o = kMaxSlices / 2; o > 0; o >>= 1) {
@@ -937,6 +980,7 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) ssd_stats_kernel(const _
     }
     if (lane == 0) {
       sm.MP = mp; sm.SP = sp; sm.MQ = mq; sm.SQ = sq; sm.argP = ap; sm.argQ = aq;
+      sm.xdP = xp; sm.xdQ = xq;
       sm.cand_off[S] = total;
       sm.n_total = total;
       sm.tmo = anyto ? 1 : 0;
@@ -1011,8 +1055,7 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) ssd_stats_kernel(const _
       acc = (d == sm.argP) ? 1.f : 0.f;
       rejected = d != sm.argP;
     } else {
-      const float xdP = Elem<TIn>::at(baseP + rbP, d);
-      const float xdQ = Elem<TIn>::at(baseQ + rbQ, d);
+      const float xdP = sm.xdP, xdQ = sm.xdQ;
       const float pd = ex2(fmaf(xdP, cT, nmP)) / SP;
       const float qd = ex2(fmaf(xdQ, cT, nmQ)) / SQ;
       const bool inS = want_topf && (xdQ > bx || (xdQ == bx && d <= bi));
@@ -1054,37 +1097,58 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) ssd_stats_kernel(const _
     a.ustate[u] = st;
     a.arrive1[u] = 0;
   }
-  __threadfence();
   __syncthreads();
-  if (tid == 0) sm.is_last_row = atomicAdd(a.row_arrive + b, 1) == upr - 1;
+  if (tid == 0) sm.is_last_row = arrive_acq_rel_gpu(a.row_arrive + b) == upr - 1;
   __syncthreads();
   if (!sm.is_last_row) return;
-  __threadfence();
 
   // =============== the row's decision: the last unit of the row to finish ===========
-  if (tid == 0) {
+  // One warp; lane k reads unit k's record (k = 32 only when K = 32), so the
+  // whole row costs one round trip.
+  if (warp == 0) {
     const UnitState* us = a.ustate + static_cast<long long>(b) * (K + 1);
     int fl = 0;
-    for (int k = 0; k < upr; ++k) fl |= __ldcg(&us[k].flags);
+    if (lane < upr) fl |= __ldcg(&us[lane].flags);
+    if (lane + 32 < upr) fl |= __ldcg(&us[lane + 32].flags);
+    fl = static_cast<int>(__reduce_or_sync(0xFFFFFFFFu, static_cast<unsigned>(fl)));
     if (verify) {
-      int kstar = K;
-      float am = INFINITY;
-      for (int k = 0; k < K; ++k) {
-        am = fminf(am, __ldcg(&us[k].amargin));
-        if (__ldcg(&us[k].rejected)) { kstar = k; break; }
+      // k* = the first rejected position, else K
+      const bool rej = lane < K && __ldcg(&us[lane].rejected) != 0;
+      const float am_l = lane < K ? __ldcg(&us[lane].amargin) : INFINITY;
+      RowState mine = {};
+      if (lane < upr) {
+        const UnitState* uk = us + lane;
+        mine.Fj = __ldcg(&uk->Fj);
+        mine.MP = __ldcg(&uk->MP); mine.SP = __ldcg(&uk->SP); mine.MQ = __ldcg(&uk->MQ); mine.SQ = __ldcg(&uk->SQ);
+        mine.Z = __ldcg(&uk->Z); mine.bx = __ldcg(&uk->bx); mine.bi = __ldcg(&uk->bi); mine.argP = __ldcg(&uk->argP);
       }
-      const UnitState* uk = us + kstar;
+      const unsigned rm = __ballot_sync(0xFFFFFFFFu, rej);
+      const int kstar = rm ? __ffs(rm) - 1 : K;
+      // the margins of the tests up to and including the first rejection
+      float am = lane <= kstar ? am_l : INFINITY;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) am = fminf(am, __shfl_xor_sync(0xFFFFFFFFu, am, o));
+      const int src = kstar & 31;
       RowState rs;
       rs.kstar = kstar;
       rs.flags = fl;
       rs.amargin = am;
-      rs.Fj = __ldcg(&uk->Fj);
-      rs.MP = __ldcg(&uk->MP); rs.SP = __ldcg(&uk->SP); rs.MQ = __ldcg(&uk->MQ); rs.SQ = __ldcg(&uk->SQ);
-      rs.Z = __ldcg(&uk->Z); rs.bx = __ldcg(&uk->bx); rs.bi = __ldcg(&uk->bi); rs.argP = __ldcg(&uk->argP);
-      a.rstate[b] = rs;
-      __threadfence();
-      st_release_gpu(a.rflag + b, static_cast<int32_t>(*reinterpret_cast<volatile uint32_t*>(a.epoch) + 1u));
-    } else {
+      rs.Fj = __shfl_sync(0xFFFFFFFFu, mine.Fj, src);
+      rs.MP = __shfl_sync(0xFFFFFFFFu, mine.MP, src); rs.SP = __shfl_sync(0xFFFFFFFFu, mine.SP, src);
+      rs.MQ = __shfl_sync(0xFFFFFFFFu, mine.MQ, src); rs.SQ = __shfl_sync(0xFFFFFFFFu, mine.SQ, src);
+      rs.Z = __shfl_sync(0xFFFFFFFFu, mine.Z, src); rs.bx = __shfl_sync(0xFFFFFFFFu, mine.bx, src);
+      rs.bi = __shfl_sync(0xFFFFFFFFu, mine.bi, src); rs.argP = __shfl_sync(0xFFFFFFFFu, mine.argP, src);
+      if (lane == 0) {
+        if (kstar >= 32) {  // K = 32, every draft accepted: unit 32 is past the warp
+          const UnitState* uk = us + kstar;
+          rs.Fj = __ldcg(&uk->Fj);
+          rs.MP = __ldcg(&uk->MP); rs.SP = __ldcg(&uk->SP); rs.MQ = __ldcg(&uk->MQ); rs.SQ = __ldcg(&uk->SQ);
+          rs.Z = __ldcg(&uk->Z); rs.bx = __ldcg(&uk->bx); rs.bi = __ldcg(&uk->bi); rs.argP = __ldcg(&uk->argP);
+        }
+        a.rstate[b] = rs;
+        st_release_gpu(a.rflag + b, static_cast<int32_t>(*reinterpret_cast<volatile uint32_t*>(a.epoch) + 1u));
+      }
+    } else if (lane == 0) {
       const bool pbad = (fl & SSD_ROW_BAD_PLAN) != 0;
       int off = 0;
       a.offsets[static_cast<long long>(b) * (K + 2)] = 0;
@@ -1098,12 +1162,11 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) ssd_stats_kernel(const _
         rs.flags = fl;
         rs.amargin = INFINITY;
         a.rstate[b] = rs;
-        __threadfence();
         const int32_t want = static_cast<int32_t>(*reinterpret_cast<volatile uint32_t*>(a.epoch) + 1u);
         for (int k = 0; k < K; ++k) st_release_gpu(a.rflag + static_cast<long long>(b) * K + k, want);
       }
     }
-    a.row_arrive[b] = 0;
+    if (lane == 0) a.row_arrive[b] = 0;
   }
 }
 
@@ -1173,14 +1236,21 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) ssd_draw_kernel(const __
     const uint32_t epoch = *reinterpret_cast<volatile const uint32_t*>(a.epoch);
     sm.dep_ok = wait_flag(a.rflag + du, static_cast<int32_t>(epoch + 1u), kDepWaitNs) ? 1 : 0;
     if (!sm.dep_ok) atomicExch(a.error, 1);
-    if (atomicAdd(a.k2_done, 1) == static_cast<int>(gridDim.x) - 1) {  // every CTA has read the epoch
+  }
+  // The row's fan-out plan depends on the inputs only: form it while the
+  // decision is awaited.
+  if (warp == 1 && (a.F != nullptr || a.alpha != nullptr)) load_plan(a, verify ? du : du / K, sm.s_F, lane);
+  __syncthreads();
+  const bool dep_ok = sm.dep_ok != 0;
+  // This CTA has read the epoch; the last CTA to do so advances it for the
+  // next call (off the path of threads 0..63, which start the stream).
+  if (tid == 2 * 32) {
+    if (atomicAdd(a.k2_done, 1) == static_cast<int>(gridDim.x) - 1) {
       *a.k2_done = 0;
       __threadfence();
       atomicAdd(a.epoch, 1u);
     }
   }
-  __syncthreads();
-  const bool dep_ok = sm.dep_ok != 0;
 
   // ---- which unit this row (or draft position) draws from ----------------------------
   int b, j, rowflags = 0, draw;
@@ -1253,6 +1323,7 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) ssd_draw_kernel(const __
                               : __ldg(a.uniforms + static_cast<long long>(b) * K + j);
   int tmo = 0;
   DrawPart* dparts = a.dparts + static_cast<long long>(du) * S;
+  int32_t seg_tok0 = -1, seg_tok1 = -1;  // the last slice: cache segment k*, prefetched
 
   if (streams) {
     // ---- this slice's mass per (chunk, warp), in token order ------------------------
@@ -1290,15 +1361,31 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) ssd_draw_kernel(const __
       dparts[slice].rs[i / kWarps][i % kWarps] = sm.rs[i / kWarps][i % kWarps];
       dparts[slice].ps[i / kWarps][i % kWarps] = sm.ps[i / kWarps][i % kWarps];
     }
-    __threadfence();
     __syncthreads();
     if constexpr (kAligned) ring.drain(tid, tmo);
-    if (tid == 0) sm.is_last = atomicAdd(a.draw_arrive + du, 1) == S - 1;
+    if (tid == 0) sm.is_last = arrive_acq_rel_gpu(a.draw_arrive + du) == S - 1;
     __syncthreads();
     if (!sm.is_last) return;
-    __threadfence();
 
     // ============ the draw: the last slice of this unit to arrive ====================
+    // Every slice's (chunk, warp) partial sums in one round trip, into the
+    // idle ring; the row's cache segment k* alongside.
+    const int nchm = ((a.d_chunk + VE - 1) / VE + kChunkVecs - 1) / kChunkVecs;  // chunks of a full slice
+    float* const Lrs = reinterpret_cast<float*>(ring_buf);
+    float* const Lps = Lrs + S * nchm * kWarps;
+    for (int i = tid; i < S * nchm * kWarps; i += kThreads) {
+      const int s2 = i / (nchm * kWarps), cw = i - s2 * (nchm * kWarps);
+      Lrs[i] = __ldcg(&dparts[s2].rs[cw / kWarps][cw % kWarps]);  // past a short slice's chunks: never read
+      Lps[i] = __ldcg(&dparts[s2].ps[cw / kWarps][cw % kWarps]);
+    }
+    if (verify && a.c_tokens && !row_invalid) {
+      int off = 0;
+      for (int k = 0; k < j; ++k) off += sm.s_F[k];
+      const int32_t* seg = a.c_tokens + static_cast<long long>(b) * a.budget + off;
+      const int Fk = sm.s_F[j];
+      if (tid < Fk) seg_tok0 = __ldcg(seg + tid);
+      if (tid + kThreads < Fk) seg_tok1 = __ldcg(seg + tid + kThreads);
+    }
     if (warp == 0) {
       float rp = 0.f, pp = 0.f;
       int to = 0;
@@ -1338,7 +1425,7 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) ssd_draw_kernel(const __
     if (warp == 0) {
       const int s_star = sm.cstar;
       const bool use_p = sm.use_p != 0;
-      const DrawPart* dp = &dparts[s_star];
+      const float* Ls = (use_p ? Lps : Lrs) + s_star * nchm * kWarps;
       const int e0s = s_star * a.d_chunk;
       const int e1s = min(V, e0s + a.d_chunk);
       const int nvs = (max(0, e1s - e0s) + VE - 1) / VE;
@@ -1347,7 +1434,7 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) ssd_draw_kernel(const __
       // chunk level: lane c holds chunk c's total
       float my = 0.f;
       if (lane < nchs) {
-        for (int w = 0; w < kWarps; ++w) my += use_p ? __ldcg(&dp->ps[lane][w]) : __ldcg(&dp->rs[lane][w]);
+        for (int w = 0; w < kWarps; ++w) my += Ls[lane * kWarps + w];
       }
       float run = 0.f, pre_k = 0.f, pre_last = 0.f;
       int k_star = -1, k_last = 0;
@@ -1360,7 +1447,7 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) ssd_draw_kernel(const __
       if (k_star < 0) { k_star = k_last; pre_k = pre_last; }
       const float tl2 = tl - pre_k;
       float mw = 0.f;
-      if (lane < kWarps) mw = use_p ? __ldcg(&dp->ps[k_star][lane]) : __ldcg(&dp->rs[k_star][lane]);
+      if (lane < kWarps) mw = Ls[k_star * kWarps + lane];
       run = 0.f;
       float pre_w = 0.f;
       pre_last = 0.f;
@@ -1425,7 +1512,6 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) ssd_draw_kernel(const __
     }
     __syncthreads();
   }
-  if (warp == 0 && (a.F != nullptr || a.alpha != nullptr)) load_plan(a, b, sm.s_F, lane);
   __syncthreads();
 
   // ============ finishing the row (verify) or the draft position (reweight) ===========
@@ -1437,10 +1523,8 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) ssd_draw_kernel(const __
       UnitState* us = a.ustate + u;
       us->dmargin = sm.margin;
       if (tmo_all) us->flags = st.flags | kFlagTimeout;
-      __threadfence();
-      sm.is_last_row = atomicAdd(a.row_arrive2 + b, 1) == K - 1;
+      sm.is_last_row = arrive_acq_rel_gpu(a.row_arrive2 + b) == K - 1;
       if (sm.is_last_row) {
-        __threadfence();
         int fl = __ldcg(&a.rstate[b].flags);
         for (int k = 0; k < K; ++k) {
           const UnitState* uk = a.ustate + static_cast<long long>(b) * (K + 1) + k;
@@ -1491,9 +1575,14 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) ssd_draw_kernel(const __
       // the key (k*, bonus) in segment k* of the row's cache
       int off = 0;
       for (int k = 0; k < kstar; ++k) off += sm.s_F[k];
-      const int32_t* seg = a.c_tokens + static_cast<long long>(b) * a.budget + off;
-      for (int i = tid; i < sm.s_F[kstar]; i += kThreads)
-        if (__ldcg(seg + i) == sm.drawn) sm.slot = off + i;
+      if (streams) {  // the segment was prefetched with the partial sums
+        if (seg_tok0 == sm.drawn) sm.slot = off + tid;
+        if (seg_tok1 == sm.drawn) sm.slot = off + tid + kThreads;
+      } else {
+        const int32_t* seg = a.c_tokens + static_cast<long long>(b) * a.budget + off;
+        for (int i = tid; i < sm.s_F[kstar]; i += kThreads)
+          if (__ldcg(seg + i) == sm.drawn) sm.slot = off + i;
+      }
     }
     __syncthreads();
     const int slot = sm.slot;
