@@ -92,6 +92,12 @@ __device__ __forceinline__ void st_release_gpu(int32_t* p, int32_t v) {
 // whole CTA wrote before the barrier (the barrier orders those writes before
 // this thread's), and after the next barrier the acquire makes what the
 // earlier arrivals published visible to the whole CTA.  Returns the old value.
+// Fire-and-forget arrival with release semantics (same publication rule as
+// above); the thread does not wait for the counter's value.
+__device__ __forceinline__ void arrive_release_gpu(int32_t* p) {
+  asm volatile("red.release.gpu.global.add.s32 [%0], 1;" ::"l"(p) : "memory");
+}
+
 __device__ __forceinline__ int32_t arrive_acq_rel_gpu(int32_t* p) {
   int32_t old;
   asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], 1;" : "=r"(old) : "l"(p) : "memory");
@@ -108,7 +114,7 @@ __device__ __forceinline__ bool wait_flag(const int32_t* flag, int32_t want, uns
     if (ld_acquire_gpu(flag) == want) return true;
     if (global_ns() - t0 > limit_ns) return false;
     __nanosleep(sleep_ns);
-    if (sleep_ns < 1024) sleep_ns <<= 1;
+    if (sleep_ns < 256) sleep_ns <<= 1;
   }
   return false;
 }
@@ -147,6 +153,34 @@ __device__ __forceinline__ float ex2(float x) {
 }
 
 // max with NaN propagation (a NaN anywhere makes the result NaN).
+// Two fp32 values in one 64-bit register pair, for the packed fp32x2
+// arithmetic of sm_100 (one instruction does both lanes, each lane rounded
+// exactly like its scalar counterpart).
+typedef unsigned long long f32x2;
+__device__ __forceinline__ f32x2 f2_pack(float lo, float hi) {
+  f32x2 r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2_unpack(f32x2 v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ f32x2 f2_fma(f32x2 a, f32x2 b, f32x2 c) {
+  f32x2 d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ f32x2 f2_add(f32x2 a, f32x2 b) {
+  f32x2 d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ f32x2 f2_mul(f32x2 a, f32x2 b) {
+  f32x2 d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+
 __device__ __forceinline__ float fmax_nan(float a, float b) {
   float d;
   asm("max.NaN.f32 %0, %1, %2;" : "=f"(d) : "f"(a), "f"(b));

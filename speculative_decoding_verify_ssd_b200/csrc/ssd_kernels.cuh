@@ -210,8 +210,8 @@ __device__ __forceinline__ void load_group(const TIn* __restrict__ base, long lo
 // maximum m, the sum s of exp2((x - m) c) rescaled when m grows, and
 // nmc = -m c.  Greedy: the running maximum and the lowest id holding it.
 template <bool kGreedy>
-__device__ __forceinline__ float consume_bf16(const uint4 w, int vbase, float c, float& m, float& s, float& nmc,
-                                              int& arg, int& nan_seen) {
+__device__ __forceinline__ float consume_bf16(const uint4 w, int vbase, float c, f32x2 c2, float& m, f32x2& s2,
+                                              f32x2& nm2, int& arg, int& nan_seen) {
   const uint32_t m2 = bf16x2_max_nan(bf16x2_max_nan(w.x, w.y), bf16x2_max_nan(w.z, w.w));
   const float vmax = fmax_nan(bf16_lo(m2), bf16_hi(m2));
   if constexpr (kGreedy) {
@@ -227,15 +227,21 @@ __device__ __forceinline__ float consume_bf16(const uint4 w, int vbase, float c,
   } else {
     if (!(vmax <= m)) {  // a new maximum (or a NaN, which then sticks)
       const float nm = fmax_nan(m, vmax);
-      s = (m == -INFINITY) ? 0.f : s * ex2((m - nm) * c);
+      const float sc = (m == -INFINITY) ? 0.f : ex2((m - nm) * c);  // s2 is 0 while m = -inf
+      s2 = f2_mul(s2, f2_pack(sc, sc));
       m = nm;
-      nmc = -m * c;
+      const float nmc = -m * c;
+      nm2 = f2_pack(nmc, nmc);
     }
-    const float e0 = ex2(fmaf(bf16_lo(w.x), c, nmc)) + ex2(fmaf(bf16_hi(w.x), c, nmc));
-    const float e1 = ex2(fmaf(bf16_lo(w.y), c, nmc)) + ex2(fmaf(bf16_hi(w.y), c, nmc));
-    const float e2 = ex2(fmaf(bf16_lo(w.z), c, nmc)) + ex2(fmaf(bf16_hi(w.z), c, nmc));
-    const float e3 = ex2(fmaf(bf16_lo(w.w), c, nmc)) + ex2(fmaf(bf16_hi(w.w), c, nmc));
-    s += (e0 + e1) + (e2 + e3);
+    // two lanes per instruction: lane 0 sums the even tokens, lane 1 the odd
+    float a0, a1, a2, a3, a4, a5, a6, a7;
+    f2_unpack(f2_fma(f2_pack(bf16_lo(w.x), bf16_hi(w.x)), c2, nm2), a0, a1);
+    f2_unpack(f2_fma(f2_pack(bf16_lo(w.y), bf16_hi(w.y)), c2, nm2), a2, a3);
+    f2_unpack(f2_fma(f2_pack(bf16_lo(w.z), bf16_hi(w.z)), c2, nm2), a4, a5);
+    f2_unpack(f2_fma(f2_pack(bf16_lo(w.w), bf16_hi(w.w)), c2, nm2), a6, a7);
+    const f32x2 e01 = f2_pack(ex2(a0), ex2(a1)), e23 = f2_pack(ex2(a2), ex2(a3));
+    const f32x2 e45 = f2_pack(ex2(a4), ex2(a5)), e67 = f2_pack(ex2(a6), ex2(a7));
+    s2 = f2_add(s2, f2_add(f2_add(e01, e23), f2_add(e45, e67)));
   }
   return vmax;
 }
@@ -707,6 +713,8 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) ssd_stats_kernel(const _
 
   // ---- the stream: online max / exp-sum (or greedy argmax) of both rows ----------
   float mP = -INFINITY, sP = 0.f, nmP1 = 0.f, mQ = -INFINITY, sQ = 0.f, nmQ1 = 0.f;
+  f32x2 sP2 = 0ull, sQ2 = 0ull, nmP2 = 0ull, nmQ2 = 0ull;  // packed (even, odd) sums and -m*c: bf16 path
+  const f32x2 cT2 = f2_pack(cT, cT);
   int argP = INT_MAX, argQ = INT_MAX, nan_seen = 0, tmo = 0;
   float vm1 = -INFINITY, vm2 = -INFINITY, vm3 = -INFINITY;  // top three vector maxima of the source row
   int g1 = -1, g2 = -1;
@@ -724,9 +732,9 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) ssd_stats_kernel(const _
       if constexpr (kAligned && sizeof(TIn) == 2) {
         float vp = -INFINITY;
         uint4 wq = make_uint4(0u, 0u, 0u, 0u), wp = wq;
-        if (hasP) { wp = ring.vec(c, slotP, t); vp = consume_bf16<kGreedy>(wp, vbase, cT, mP, sP, nmP1, argP, nan_seen); }
+        if (hasP) { wp = ring.vec(c, slotP, t); vp = consume_bf16<kGreedy>(wp, vbase, cT, cT2, mP, sP2, nmP2, argP, nan_seen); }
         float vq = -INFINITY;
-        if (hasQ) { wq = ring.vec(c, slotQ, t); vq = consume_bf16<kGreedy>(wq, vbase, cT, mQ, sQ, nmQ1, argQ, nan_seen); }
+        if (hasQ) { wq = ring.vec(c, slotQ, t); vq = consume_bf16<kGreedy>(wq, vbase, cT, cT2, mQ, sQ2, nmQ2, argQ, nan_seen); }
         vsrc = srcQ ? vq : vp;
         wsrc = srcQ ? wq : wp;
       } else {
@@ -760,6 +768,12 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) ssd_stats_kernel(const _
   }
   if constexpr (kGreedy) {
     if (nan_seen) { mP = __int_as_float(0x7FC00000); mQ = mP; }
+  } else if constexpr (kAligned && sizeof(TIn) == 2) {
+    float lo, hi;
+    f2_unpack(sP2, lo, hi);
+    sP = lo + hi;
+    f2_unpack(sQ2, lo, hi);
+    sQ = lo + hi;
   }
   // The slice that holds the drafted token reads its two logits for the
   // unit's accept test now (this CTA has just streamed them through L2).
@@ -918,9 +932,19 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) ssd_stats_kernel(const _
   }
   __syncthreads();
   if constexpr (kAligned) ring.drain(tid, tmo);
-  if (tid == 0) sm.is_last = arrive_acq_rel_gpu(a.arrive1 + u) == S - 1;
+  // The unit's last slice, the last of its CTAs to be scheduled, finalizes:
+  // the others publish and leave without waiting; it waits (bounded) until
+  // they have all published.
+  if (slice != S - 1) {
+    if (tid == 0) arrive_release_gpu(a.arrive1 + u);
+    return;
+  }
+  if (tid == 0) {
+    sm.is_last = wait_flag(a.arrive1 + u, S - 1, kDepWaitNs) ? 1 : 0;
+    if (!sm.is_last) atomicExch(a.error, 1);
+  }
   __syncthreads();
-  if (!sm.is_last) return;
+  const bool arrivals_ok = sm.is_last != 0;
 
   // =============== the unit's finalizer: the last slice to arrive ===================
   const SlicePart* parts = a.parts + u * S;
@@ -989,7 +1013,7 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) ssd_stats_kernel(const _
   }
   __syncthreads();
   const float MP = sm.MP, MQ = sm.MQ, SP = sm.SP, SQ = sm.SQ;
-  if (sm.tmo) flags |= kFlagTimeout;
+  if (sm.tmo || !arrivals_ok) flags |= kFlagTimeout;
   if (hasP && !(MP > -INFINITY && MP < INFINITY)) flags |= SSD_ROW_NONFINITE;
   if (hasQ && !(MQ > -INFINITY && MQ < INFINITY)) flags |= SSD_ROW_NONFINITE;
   const bool valid = (flags & SSD_ROW_INVALID) == 0;
@@ -1098,9 +1122,18 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) ssd_stats_kernel(const _
     a.arrive1[u] = 0;
   }
   __syncthreads();
-  if (tid == 0) sm.is_last_row = arrive_acq_rel_gpu(a.row_arrive + b) == upr - 1;
+  // Likewise per row: unit j = 0, whose CTAs are the row's last to be
+  // scheduled, decides once the other units have published.
+  if (j != 0) {
+    if (tid == 0) arrive_release_gpu(a.row_arrive + b);
+    return;
+  }
+  if (tid == 0) {
+    sm.is_last_row = wait_flag(a.row_arrive + b, upr - 1, kDepWaitNs) ? 1 : 0;
+    if (!sm.is_last_row) atomicExch(a.error, 1);
+  }
   __syncthreads();
-  if (!sm.is_last_row) return;
+  const bool row_ok = sm.is_last_row != 0;
 
   // =============== the row's decision: the last unit of the row to finish ===========
   // One warp; lane k reads unit k's record (k = 32 only when K = 32), so the
@@ -1111,6 +1144,7 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) ssd_stats_kernel(const _
     if (lane < upr) fl |= __ldcg(&us[lane].flags);
     if (lane + 32 < upr) fl |= __ldcg(&us[lane + 32].flags);
     fl = static_cast<int>(__reduce_or_sync(0xFFFFFFFFu, static_cast<unsigned>(fl)));
+    if (!row_ok) fl |= kFlagTimeout;
     if (verify) {
       // k* = the first rejected position, else K
       const bool rej = lane < K && __ldcg(&us[lane].rejected) != 0;
