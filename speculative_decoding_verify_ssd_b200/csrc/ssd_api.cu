@@ -199,11 +199,11 @@ static WsLayout ws_layout(int B, int K, int V, int dtype) {
   w.ustate = off;      off = up256(off + units * sizeof(UnitState));
   w.dparts = off;      off = up256(off + nb * static_cast<size_t>(K) * ns * sizeof(DrawPart));
   w.rstate = off;      off = up256(off + nb * sizeof(RowState));
+  w.rflag = off;       off += nb * static_cast<size_t>(K) * sizeof(uint64_t);  // 8-byte aligned here
   w.arrive1 = off;     off += units * sizeof(int32_t);
   w.row_arrive = off;  off += nb * sizeof(int32_t);
   w.draw_arrive = off; off += nb * static_cast<size_t>(K) * sizeof(int32_t);
   w.row_arrive2 = off; off += nb * sizeof(int32_t);
-  w.rflag = off;       off += nb * static_cast<size_t>(K) * sizeof(int32_t);
   w.epoch = off;       off += sizeof(uint32_t);
   w.k2_done = off;     off += sizeof(int32_t);
   w.error = off;       off += sizeof(int32_t);
@@ -221,7 +221,7 @@ static void bind_workspace(Args& a, void* ws, const WsLayout& w) {
   a.row_arrive = reinterpret_cast<int32_t*>(base + w.row_arrive);
   a.draw_arrive = reinterpret_cast<int32_t*>(base + w.draw_arrive);
   a.row_arrive2 = reinterpret_cast<int32_t*>(base + w.row_arrive2);
-  a.rflag = reinterpret_cast<int32_t*>(base + w.rflag);
+  a.rflag = reinterpret_cast<uint64_t*>(base + w.rflag);
   a.epoch = reinterpret_cast<uint32_t*>(base + w.epoch);
   a.k2_done = reinterpret_cast<int32_t*>(base + w.k2_done);
   a.error = reinterpret_cast<int32_t*>(base + w.error);

@@ -105,6 +105,34 @@ __device__ __forceinline__ int32_t arrive_acq_rel_gpu(int32_t* p) {
 }
 
 
+__device__ __forceinline__ uint64_t ld_acquire_gpu_u64(const uint64_t* p) {
+  uint64_t v;
+  asm volatile("ld.acquire.gpu.global.b64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ void st_release_gpu_u64(uint64_t* p, uint64_t v) {
+  asm volatile("st.release.gpu.global.b64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+
+// Bounded wait for a 64-bit word whose high half is a tag: true (and the
+// word in *out) once the high half equals `tag`; false after `limit_ns`.
+__device__ __forceinline__ bool wait_tagged(const uint64_t* word, uint32_t tag, unsigned long long limit_ns,
+                                            uint64_t* out) {
+  const unsigned long long t0 = global_ns();
+  uint32_t sleep_ns = 64;
+  for (uint32_t i = 0; i < 50000000u; ++i) {
+    const uint64_t v = ld_acquire_gpu_u64(word);
+    if (static_cast<uint32_t>(v >> 32) == tag) {
+      *out = v;
+      return true;
+    }
+    if (global_ns() - t0 > limit_ns) return false;
+    __nanosleep(sleep_ns);
+    if (sleep_ns < 256) sleep_ns <<= 1;
+  }
+  return false;
+}
+
 // Bounded wait for a flag written by another CTA (or grid): true once
 // *flag == want; false after `limit_ns` of waiting (or as many polls).
 __device__ __forceinline__ bool wait_flag(const int32_t* flag, int32_t want, unsigned long long limit_ns) {

@@ -156,7 +156,7 @@ struct Args {
   int32_t* row_arrive;
   int32_t* draw_arrive;
   int32_t* row_arrive2;
-  int32_t* rflag;          // per draw unit: epoch + 1 once the row decision is written
+  uint64_t* rflag;         // per draw unit, once the row decision is written: (epoch + 1) << 32 | k* << 8 | flags
   uint32_t* epoch;         // calls completed on this workspace (kernel 2 advances it)
   int32_t* k2_done;        // kernel 2 CTAs past their wait
   int32_t* error;
@@ -1180,7 +1180,9 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) ssd_stats_kernel(const _
           rs.Z = __ldcg(&uk->Z); rs.bx = __ldcg(&uk->bx); rs.bi = __ldcg(&uk->bi); rs.argP = __ldcg(&uk->argP);
         }
         a.rstate[b] = rs;
-        st_release_gpu(a.rflag + b, static_cast<int32_t>(*reinterpret_cast<volatile uint32_t*>(a.epoch) + 1u));
+        const uint64_t tag = *reinterpret_cast<volatile uint32_t*>(a.epoch) + 1u;
+        st_release_gpu_u64(a.rflag + b, tag << 32 | static_cast<uint64_t>(kstar) << 8 |
+                                            static_cast<uint64_t>(fl & 0xFF));
       }
     } else if (lane == 0) {
       const bool pbad = (fl & SSD_ROW_BAD_PLAN) != 0;
@@ -1196,8 +1198,9 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) ssd_stats_kernel(const _
         rs.flags = fl;
         rs.amargin = INFINITY;
         a.rstate[b] = rs;
-        const int32_t want = static_cast<int32_t>(*reinterpret_cast<volatile uint32_t*>(a.epoch) + 1u);
-        for (int k = 0; k < K; ++k) st_release_gpu(a.rflag + static_cast<long long>(b) * K + k, want);
+        const uint64_t tag = *reinterpret_cast<volatile uint32_t*>(a.epoch) + 1u;
+        for (int k = 0; k < K; ++k)
+          st_release_gpu_u64(a.rflag + static_cast<long long>(b) * K + k, tag << 32 | static_cast<uint64_t>(fl & 0xFF));
       }
     }
     if (lane == 0) a.row_arrive[b] = 0;
@@ -1207,7 +1210,7 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) ssd_stats_kernel(const _
 // Shared memory of kernel 2.
 struct Smem2 {
   uint64_t full[kStages];
-  int32_t dep_ok;
+  int32_t dep_ok, w_kstar, w_flags;
   float rs[kMaxChunks][kWarps];
   float ps[kMaxChunks][kWarps];
   int32_t s_F[SSD_MAX_K + 1];
@@ -1268,8 +1271,11 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) ssd_draw_kernel(const __
   // ---- the row decision this CTA needs (kernel 1 may still be running) -------------
   if (tid == 0) {
     const uint32_t epoch = *reinterpret_cast<volatile const uint32_t*>(a.epoch);
-    sm.dep_ok = wait_flag(a.rflag + du, static_cast<int32_t>(epoch + 1u), kDepWaitNs) ? 1 : 0;
+    uint64_t word = 0;
+    sm.dep_ok = wait_tagged(a.rflag + du, epoch + 1u, kDepWaitNs, &word) ? 1 : 0;
     if (!sm.dep_ok) atomicExch(a.error, 1);
+    sm.w_kstar = static_cast<int32_t>((word >> 8) & 0xFF);  // the decision itself travels with the flag
+    sm.w_flags = static_cast<int32_t>(word & 0xFF);
   }
   // The row's fan-out plan depends on the inputs only: form it while the
   // decision is awaited.
@@ -1291,25 +1297,16 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) ssd_draw_kernel(const __
   float amargin = INFINITY;
   UnitState st;
   if (verify) {
+    // k* and the row's flags came with the flag word: the stream can start
+    // before the row's statistics are read
     b = du;
-    RowState rs;
-    rs.kstar = __ldcg(&a.rstate[b].kstar); rs.flags = __ldcg(&a.rstate[b].flags);
-    rs.amargin = __ldcg(&a.rstate[b].amargin); rs.Fj = __ldcg(&a.rstate[b].Fj);
-    rs.MP = __ldcg(&a.rstate[b].MP); rs.SP = __ldcg(&a.rstate[b].SP);
-    rs.MQ = __ldcg(&a.rstate[b].MQ); rs.SQ = __ldcg(&a.rstate[b].SQ);
-    rs.Z = __ldcg(&a.rstate[b].Z); rs.bx = __ldcg(&a.rstate[b].bx);
-    rs.bi = __ldcg(&a.rstate[b].bi); rs.argP = __ldcg(&a.rstate[b].argP);
-    if (!dep_ok || rs.kstar < 0 || rs.kstar > K) {  // the decision never came: a timed-out row
-      rs.kstar = K;
-      rs.flags = kFlagTimeout;
+    j = sm.w_kstar;
+    rowflags = sm.w_flags;
+    if (!dep_ok || j < 0 || j > K) {  // the decision never came: a timed-out row
+      j = K;
+      rowflags = kFlagTimeout;
     }
-    j = rs.kstar;
-    rowflags = rs.flags;
-    amargin = rs.amargin;
     draw = j < K ? kDrawResidual : kDrawP;
-    st.MP = rs.MP; st.SP = rs.SP; st.MQ = rs.MQ; st.SQ = rs.SQ;
-    st.Z = rs.Z; st.bx = rs.bx; st.bi = rs.bi; st.argP = rs.argP; st.argQ = 0;
-    st.Fj = rs.Fj; st.flags = rowflags;
   } else {
     b = du / K;
     j = du % K;
@@ -1346,6 +1343,15 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) ssd_draw_kernel(const __
   ring.nch = nch;
   const int slotP = 0, slotQ = useP ? 1 : 0;
   if (kAligned && streams) ring.start(tid);
+  if (verify) {  // the statistics of unit k*, while the first chunks are in flight
+    const RowState* rs = a.rstate + b;
+    amargin = __ldcg(&rs->amargin);
+    st.MP = __ldcg(&rs->MP); st.SP = __ldcg(&rs->SP); st.MQ = __ldcg(&rs->MQ); st.SQ = __ldcg(&rs->SQ);
+    st.Z = __ldcg(&rs->Z); st.bx = __ldcg(&rs->bx); st.bi = __ldcg(&rs->bi); st.argP = __ldcg(&rs->argP);
+    st.argQ = 0;
+    st.Fj = __ldcg(&rs->Fj);
+    st.flags = rowflags;
+  }
 
   const float cT = kGreedy ? 0.f : kLog2e / a.T;
   const float C = a.C;
@@ -1383,13 +1389,16 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) ssd_draw_kernel(const __
       if (lane == 0) { sm.rs[c][warp] = rsum; sm.ps[c][warp] = psum; }
     }
     tmo = __syncthreads_or(tmo);
-    if (tid == 0) {
+    if (warp == 0) {  // the slice's masses: lane l sums entries l, l + 32, ... then a butterfly
       float R = 0.f, RP = 0.f;
-      for (int c = 0; c < nch; ++c)
-        for (int w = 0; w < kWarps; ++w) { R += sm.rs[c][w]; RP += sm.ps[c][w]; }
-      dparts[slice].R = R;
-      dparts[slice].RP = RP;
-      dparts[slice].timeout = tmo;
+      for (int i = lane; i < nch * kWarps; i += 32) { R += sm.rs[i / kWarps][i % kWarps]; RP += sm.ps[i / kWarps][i % kWarps]; }
+      R = warp_sum(R);
+      RP = warp_sum(RP);
+      if (lane == 0) {
+        dparts[slice].R = R;
+        dparts[slice].RP = RP;
+        dparts[slice].timeout = tmo;
+      }
     }
     for (int i = tid; i < nch * kWarps; i += kThreads) {
       dparts[slice].rs[i / kWarps][i % kWarps] = sm.rs[i / kWarps][i % kWarps];
