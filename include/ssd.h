@@ -220,8 +220,8 @@ ssd_status ssd_cache_lookup(const int32_t* offsets, const int32_t* tokens, int B
 
 /* Workspace size in bytes for ssd_verify / ssd_saguaro_reweight at
  * (B, K, V, dtype).  The workspace holds per-slice and per-(row, position)
- * partial results, per-row states, then arrival counters and one device error
- * word.  It must be 256-byte aligned and zero-filled before its first use;
+ * partial results, per-row states, per-row decision words tagged with a call
+ * epoch, then arrival counters and one device error word.  It must be 256-byte aligned and zero-filled before its first use;
  * each completed call leaves the counters zero again, so it can be reused by
  * the next call on the same stream (calls that overlap on the GPU must not
  * share one).  0 for invalid sizes. */
@@ -229,7 +229,9 @@ size_t ssd_workspace_bytes(int B, int K, int V, int dtype);
 
 /* Reads and clears the device error word of a workspace laid out for
  * (B, K, V, dtype), synchronising `stream`: *out = SSD_OK, or SSD_ERR_TIMEOUT
- * when a bounded device wait of an earlier call gave up.  Not for the hot path. */
+ * when a bounded device wait of an earlier call gave up.  After a timeout the
+ * workspace's counters may be left non-zero: zero-fill it again before its
+ * next use.  Not for the hot path. */
 ssd_status ssd_read_device_error(void* workspace, int B, int K, int V, int dtype, void* stream,
                                  int32_t* out);
 
