@@ -152,11 +152,22 @@ class Workspace:
     def ptr(self):
         return C.c_void_p(self.view.data_ptr())
 
+    def reset(self):
+        """Zero-fill the workspace again (needed after a device timeout, which
+        may leave arrival counters non-zero).  Synchronises the device, so the
+        next call on any stream sees the zeros."""
+        self.view.zero_()
+        torch.cuda.synchronize(self.view.device)
+
     def device_error(self, stream=None) -> int:
+        """SSD_OK, or SSD_ERR_TIMEOUT if a bounded device wait of an earlier
+        call gave up; in that case the workspace is zero-filled again."""
         out = C.c_int32(0)
         _check(load().ssd_read_device_error(self.ptr(), self.B, self.K, self.V, self.dtype, _stream(stream),
                                             C.byref(out)),
                "ssd_read_device_error")
+        if out.value != 0:
+            self.reset()
         return out.value
 
 
