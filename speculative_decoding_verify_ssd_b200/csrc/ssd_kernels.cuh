@@ -16,20 +16,22 @@
 //       slice's share of the unit's top-F, [ZH] challenge 2 "top-F tokens")
 //       comes from registers: the F-th largest thread maximum bounds it from
 //       below.
-//   It publishes a small partial and leaves.  The last CTA of a unit to
-//   arrive (a counter, no waiting) merges the partials, selects the exact
+//   It publishes a small partial and leaves (one thread's release reduction
+//   on the unit's counter).  The unit's last slice, its last CTA to be
+//   scheduled, waits for the others, merges the partials, selects the exact
 //   top-F by (logit desc, token id asc), forms Q_S and the Saguaro normaliser
 //   Z = 1 - (1 - C) Q_S ([ZH] challenge 2; [NL] 3B), and runs the lossless
-//   accept test a_j = min(1, p_j(d_j) / q'_j(d_j)); the last unit of a row
-//   fixes k*, the first rejected position, and raises the row's flag.  Rows
-//   are taken in order, so they are decided one after another.
+//   accept test a_j = min(1, p_j(d_j) / q'_j(d_j)); in the same way unit
+//   j = 0, the row's last to be scheduled, fixes k*, the first rejected
+//   position, and publishes the row's decision word (call epoch, k*, flags).
+//   Rows are taken in order, so they are decided one after another.
 //
 // Kernel 2 (draw): one CTA per (row, slice) of the single unit each row
 //   draws from: the residual r = max(0, p_k* - q'_k*) (or p_K after full
 //   acceptance, or q' for a draft draw).  It is a programmatic dependent of
 //   kernel 1 (scheduled once every kernel-1 CTA has started) and each CTA
-//   waits only for its own row's flag, so the draws of early rows run while
-//   kernel 1 finishes.  Each CTA sums its slice of r per
+//   waits only for its own row's decision word, so the draws of early rows
+//   run while kernel 1 finishes.  Each CTA sums its slice of r per
 //   (ring chunk, warp); the last CTA of the row finds where the cumulative
 //   mass crosses u * R in token order (slice, chunk, warp, then one re-read
 //   vector per lane), draws the bonus token, and finishes the row: outputs,
@@ -946,7 +948,7 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) ssd_stats_kernel(const _
   __syncthreads();
   const bool arrivals_ok = sm.is_last != 0;
 
-  // =============== the unit's finalizer: the last slice to arrive ===================
+  // =============== the unit's finalizer: its last slice, once all have arrived ======
   const SlicePart* parts = a.parts + u * S;
   // Every slice's published candidates, loaded at once with the statistics
   // (slot c * cap + r holds candidate r of slice c; entries past a slice's
@@ -1135,7 +1137,7 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) ssd_stats_kernel(const _
   __syncthreads();
   const bool row_ok = sm.is_last_row != 0;
 
-  // =============== the row's decision: the last unit of the row to finish ===========
+  // =============== the row's decision: unit j = 0, once all units have arrived ======
   // One warp; lane k reads unit k's record (k = 32 only when K = 32), so the
   // whole row costs one round trip.
   if (warp == 0) {
@@ -1297,7 +1299,7 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) ssd_draw_kernel(const __
   float amargin = INFINITY;
   UnitState st;
   if (verify) {
-    // k* and the row's flags came with the flag word: the stream can start
+    // k* and the row's flags came with the decision word: the stream can start
     // before the row's statistics are read
     b = du;
     j = sm.w_kstar;
