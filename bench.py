@@ -356,7 +356,7 @@ def run_reference(args, rank, world):
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic", "config": workload_config(w, world),
             "cpu_baseline": {"value": value, "unit": "rows/s", "cores": cores, "kind": "oracle",
-                             "sample": f"{cores} rows of {w.name} per step"},
+                             "sample": f"{min(w.B, cores)} row{'s' if min(w.B, cores) != 1 else ''} of {w.name} per step"},
             "e2e": {"value": value, "unit": "rows/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
