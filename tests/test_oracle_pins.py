@@ -505,3 +505,55 @@ def test_expected_hit_probability_matches_frequency():
     assert np.allclose(out["p_hit"], ph)
     freq = out["hit"].mean()
     assert abs(freq - ph) < 4.5 * np.sqrt(ph * (1 - ph) / n) + 1e-9
+
+
+# ---------------------------------------------------------------------------
+# Exact boundaries of the accept test and the bonus draw.  Logits of 0 and
+# -inf make every probability dyadic, so each comparison below is exact in
+# fp32 and fp64; the expected outcomes are worked out by hand.
+# ---------------------------------------------------------------------------
+NEG = -np.inf
+
+
+def _one_row(p_logits, q_logits, d, u):
+    """K = len(q_logits), V = 4, T = 1, no reweighting."""
+    target = np.array([p_logits], dtype=np.float32)
+    draft = np.array([q_logits], dtype=np.float32)
+    return oracle.verify(target, draft, np.array([d], np.int32), np.array([u], np.float32), 1.0)
+
+
+def test_accept_test_is_strict_at_a():
+    # p_0 uniform (1/4 each), q_0 = (1/2, 1/2, 0, 0), d_0 = 0: a_0 = (1/4)/(1/2) = 1/2
+    p = [[0, 0, 0, 0], [0, 0, 0, 0]]
+    q = [[0, 0, NEG, NEG]]
+    below = _one_row(p, q, [0], [0.5 - 2.0 ** -24, 0.3])
+    at = _one_row(p, q, [0], [0.5, 0.3])
+    assert below["accept_prob"][0, 0] == 0.5 and at["accept_prob"][0, 0] == 0.5
+    assert below["n_accepted"][0] == 1          # u < a accepts
+    assert at["n_accepted"][0] == 0             # u = a rejects
+    # after the rejection: r = max(0, p - q) = (0, 0, 1/4, 1/4), R = 1/2
+    assert at["residual_mass"][0] == 0.5
+
+
+def test_bonus_inverse_cdf_is_strict_in_token_order():
+    # continuing the case above (k* = 0, r = (0, 0, 1/4, 1/4), R = 1/2):
+    # u_K R = 1/4 equals the CDF step at token 2, strict > moves past it
+    p = [[0, 0, 0, 0], [0, 0, 0, 0]]
+    q = [[0, 0, NEG, NEG]]
+    at_step = _one_row(p, q, [0], [0.5, 0.5])
+    assert at_step["bonus"][0] == 3
+    below_step = _one_row(p, q, [0], [0.5, 0.5 - 2.0 ** -24])
+    assert below_step["bonus"][0] == 2
+    assert list(at_step["out_tokens"][0]) == [3, -1]
+
+
+def test_bonus_uses_the_last_uniform_whatever_k_star():
+    # K = 2, rejection at position 0 (p_0(d_0) = 0): r = p_0 = (1/2, 1/2, 0, 0),
+    # R = 1.  The bonus takes u_K = u_2 = 1/2 -> strict > gives token 1; u_1
+    # (0.1, unused) would have given token 0.
+    p = [[0, 0, NEG, NEG], [0, 0, 0, 0], [0, 0, 0, 0]]
+    q = [[NEG, NEG, 0, 0], [0, 0, 0, 0]]
+    out = _one_row(p, q, [2, 0], [0.25, 0.1, 0.5])
+    assert out["n_accepted"][0] == 0 and out["accept_prob"][0, 0] == 0.0
+    assert out["residual_mass"][0] == 1.0
+    assert out["bonus"][0] == 1
