@@ -173,11 +173,17 @@ ssd_status ssd_verify(const void* target_logits, const void* draft_logits, const
  *   SSD_NOALLOC_MAX_WORKSPACE (16 MiB, enough for B=64, K=6, V=128256 bf16);
  *   larger problems return SSD_ERR_WORKSPACE before touching the device.
  *   First call on a device: looks up the buffer's device address
- *   (cudaGetSymbolAddress, with that device current) and zero-fills it with a
- *   synchronous memset; make that first call before any stream capture.
- *   Later calls only launch.  The buffer is one per device: calls that
- *   overlap on one device (two streams, or two host threads) share it and
- *   race; serialise them.  Each completed call leaves its counters zero.
+ *   (cudaGetSymbolAddress, with that device current); make that first call
+ *   before any stream capture.  Every call then enqueues, on `stream` and
+ *   ahead of its kernels, a cudaMemsetAsync that zeroes the part of the
+ *   buffer holding this shape's arrival counters, decision words, epoch and
+ *   error word (a few KB).  So a call never depends on the shape of the call
+ *   before it, nor on whether that call timed out.  Device timeouts are
+ *   reported through the rows' SSD_ROW_DEVICE_TIMEOUT bits only: the
+ *   buffer's error word is cleared by the next call.
+ *   The buffer is one per device, and the current device must own every
+ *   pointer passed.  Calls that overlap on one device (two streams, or two
+ *   host threads) share the buffer and race: serialise them.
  */
 #define SSD_NOALLOC_MAX_WORKSPACE (16u << 20)
 ssd_status ssd_verify_noalloc(const void* target_logits, const void* draft_logits, const void* draft_next,

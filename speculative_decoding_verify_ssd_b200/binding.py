@@ -171,6 +171,22 @@ class Workspace:
         return out.value
 
 
+_default_ws = {}
+
+
+def default_workspace(device, B: int, K: int, V: int, dtype: int) -> Workspace:
+    """The workspace used when a call passes none: one per (device, B, K, V,
+    dtype), made on first use and kept, so repeated calls of one shape do not
+    allocate.  Calls that share it must not overlap on the GPU (one stream);
+    calls on several streams pass a Workspace each."""
+    key = (torch.device(device).index, B, K, V, dtype)
+    ws = _default_ws.get(key)
+    if ws is None:
+        ws = Workspace(B, K, device, V, dtype)
+        _default_ws[key] = ws
+    return ws
+
+
 def ssd_fanout_plan(alpha: torch.Tensor, K: int, budget: int, mode: int = FANOUT_GEOMETRIC,
                     F: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
     B = alpha.shape[0]
@@ -178,8 +194,9 @@ def ssd_fanout_plan(alpha: torch.Tensor, K: int, budget: int, mode: int = FANOUT
     if F is None:
         F = torch.empty((B, K + 1), dtype=torch.int32, device=alpha.device)
     _need(F, "F", torch.int32, (B, K + 1), alpha.device)
-    _check(load().ssd_fanout_plan(_ptr(alpha), B, K, budget, mode, _ptr(F), _stream(stream)),
-           "ssd_fanout_plan")
+    with torch.cuda.device(alpha.device):
+        _check(load().ssd_fanout_plan(_ptr(alpha), B, K, budget, mode, _ptr(F), _stream(stream)),
+               "ssd_fanout_plan")
     return F
 
 
@@ -243,7 +260,7 @@ def ssd_verify(target: torch.Tensor, draft: torch.Tensor, draft_tokens: torch.Te
     if cache and F is None and alpha is None:
         raise ValueError("a cache needs a fan-out plan (F or alpha)")
     if workspace is None:
-        workspace = Workspace(B, K, dev, V, dt)
+        workspace = default_workspace(dev, B, K, V, dt)
     if out is None:
         out = alloc_verify_result(B, K, budget, dev, cache)
     cstruct = None
@@ -251,13 +268,14 @@ def ssd_verify(target: torch.Tensor, draft: torch.Tensor, draft_tokens: torch.Te
         cstruct = _Cache(out.cache_offsets.data_ptr(), out.cache_tokens.data_ptr(),
                          None if payload is None else payload.data_ptr(), out.hit.data_ptr(),
                          out.slot.data_ptr(), out.next_tokens.data_ptr(), fallback_seed)
-    code = load().ssd_verify(
-        _ptr(target), _ptr(draft), _ptr(draft_next), dt, B, K, V, _ptr(draft_tokens), _ptr(uniforms),
-        float(T), _ptr(F), _ptr(alpha), int(fanout_mode), float(C_coef), int(budget),
-        _ptr(out.n_accepted), _ptr(out.bonus),
-        _ptr(out.out_tokens), _ptr(out.accept_prob), _ptr(out.residual_mass),
-        C.byref(cstruct) if cstruct is not None else None, _ptr(out.status), workspace.ptr(),
-        workspace.nbytes, _stream(stream))
+    with torch.cuda.device(dev):
+        code = load().ssd_verify(
+            _ptr(target), _ptr(draft), _ptr(draft_next), dt, B, K, V, _ptr(draft_tokens), _ptr(uniforms),
+            float(T), _ptr(F), _ptr(alpha), int(fanout_mode), float(C_coef), int(budget),
+            _ptr(out.n_accepted), _ptr(out.bonus),
+            _ptr(out.out_tokens), _ptr(out.accept_prob), _ptr(out.residual_mass),
+            C.byref(cstruct) if cstruct is not None else None, _ptr(out.status), workspace.ptr(),
+            workspace.nbytes, _stream(stream))
     _check(code, "ssd_verify")
     return out
 
@@ -300,12 +318,13 @@ def ssd_verify_noalloc(target: torch.Tensor, draft: torch.Tensor, draft_tokens: 
         cstruct = _Cache(out.cache_offsets.data_ptr(), out.cache_tokens.data_ptr(),
                          None if payload is None else payload.data_ptr(), out.hit.data_ptr(),
                          out.slot.data_ptr(), out.next_tokens.data_ptr(), fallback_seed)
-    code = load().ssd_verify_noalloc(
-        _ptr(target), _ptr(draft), _ptr(draft_next), dt, B, K, V, _ptr(draft_tokens), _ptr(uniforms),
-        float(T), _ptr(F), _ptr(alpha), int(fanout_mode), float(C_coef), int(budget),
-        _ptr(out.n_accepted), _ptr(out.bonus),
-        _ptr(out.out_tokens), _ptr(out.accept_prob), _ptr(out.residual_mass),
-        C.byref(cstruct) if cstruct is not None else None, _ptr(out.status), _stream(stream))
+    with torch.cuda.device(dev):
+        code = load().ssd_verify_noalloc(
+            _ptr(target), _ptr(draft), _ptr(draft_next), dt, B, K, V, _ptr(draft_tokens), _ptr(uniforms),
+            float(T), _ptr(F), _ptr(alpha), int(fanout_mode), float(C_coef), int(budget),
+            _ptr(out.n_accepted), _ptr(out.bonus),
+            _ptr(out.out_tokens), _ptr(out.accept_prob), _ptr(out.residual_mass),
+            C.byref(cstruct) if cstruct is not None else None, _ptr(out.status), _stream(stream))
     _check(code, "ssd_verify_noalloc")
     return out
 
@@ -356,7 +375,7 @@ def ssd_saguaro_reweight(draft: torch.Tensor, T: float, F: torch.Tensor, C_coef:
             raise ValueError("guess rows must match the draft dtype and device")
         stride = int(guess_row_stride if guess_row_stride is not None else guess.stride(0))
     if workspace is None:
-        workspace = Workspace(B, K, dev, V, dt)
+        workspace = default_workspace(dev, B, K, V, dt)
     i32 = dict(dtype=torch.int32, device=dev)
     r = ReweightResult(topf_tokens=torch.full((B, max(budget, 1)), -2, **i32),
                        offsets=torch.empty((B, K + 2), **i32),
@@ -364,10 +383,11 @@ def ssd_saguaro_reweight(draft: torch.Tensor, T: float, F: torch.Tensor, C_coef:
                        q_lse=torch.empty((B, K), dtype=torch.float32, device=dev),
                        status=torch.empty(B, **i32),
                        draft_tokens=torch.empty((B, K), **i32) if u_draft is not None else None)
-    code = load().ssd_saguaro_reweight(
-        _ptr(draft), dt, B, K, V, float(T), _ptr(F), float(C_coef), int(budget), _ptr(guess), stride,
-        _ptr(u_draft), _ptr(r.topf_tokens), _ptr(r.offsets), _ptr(r.Z), _ptr(r.q_lse),
-        _ptr(r.draft_tokens), _ptr(r.status), workspace.ptr(), workspace.nbytes, _stream(stream))
+    with torch.cuda.device(dev):
+        code = load().ssd_saguaro_reweight(
+            _ptr(draft), dt, B, K, V, float(T), _ptr(F), float(C_coef), int(budget), _ptr(guess), stride,
+            _ptr(u_draft), _ptr(r.topf_tokens), _ptr(r.offsets), _ptr(r.Z), _ptr(r.q_lse),
+            _ptr(r.draft_tokens), _ptr(r.status), workspace.ptr(), workspace.nbytes, _stream(stream))
     _check(code, "ssd_saguaro_reweight")
     return r
 
@@ -383,8 +403,9 @@ def ssd_cache_build(F: torch.Tensor, topf_tokens: torch.Tensor, budget: int,
         _need(guess_K, "guess_K", torch.int32, (B, budget), dev)
     offsets = torch.empty((B, K + 2), dtype=torch.int32, device=dev)
     tokens = torch.empty((B, budget), dtype=torch.int32, device=dev)
-    _check(load().ssd_cache_build(_ptr(F), _ptr(topf_tokens), _ptr(guess_K), B, K, budget, _ptr(offsets),
-                                  _ptr(tokens), _stream(stream)), "ssd_cache_build")
+    with torch.cuda.device(dev):
+        _check(load().ssd_cache_build(_ptr(F), _ptr(topf_tokens), _ptr(guess_K), B, K, budget, _ptr(offsets),
+                                      _ptr(tokens), _stream(stream)), "ssd_cache_build")
     return offsets, tokens
 
 
@@ -403,7 +424,8 @@ def ssd_cache_lookup(offsets: torch.Tensor, tokens: torch.Tensor, k: torch.Tenso
     hit = torch.empty(B, dtype=torch.uint8, device=dev)
     slot = torch.empty(B, dtype=torch.int32, device=dev)
     nxt = torch.empty((B, K), dtype=torch.int32, device=dev)
-    _check(load().ssd_cache_lookup(_ptr(offsets), _ptr(tokens), B, K, budget, _ptr(k), _ptr(bonus),
-                                   _ptr(payload), fallback_seed, V, _ptr(hit), _ptr(slot), _ptr(nxt),
-                                   _stream(stream)), "ssd_cache_lookup")
+    with torch.cuda.device(dev):
+        _check(load().ssd_cache_lookup(_ptr(offsets), _ptr(tokens), B, K, budget, _ptr(k), _ptr(bonus),
+                                       _ptr(payload), fallback_seed, V, _ptr(hit), _ptr(slot), _ptr(nxt),
+                                       _stream(stream)), "ssd_cache_lookup")
     return hit, slot, nxt

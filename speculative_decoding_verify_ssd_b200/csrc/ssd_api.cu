@@ -468,8 +468,8 @@ static constexpr int kNoallocMaxDevices = 64;
 static void* g_noalloc_ptr[kNoallocMaxDevices];
 static std::mutex g_noalloc_mu;
 
-// The buffer's address on the current device; the first call per device also
-// zero-fills it (the arrival counters must start at zero) and waits for that.
+// The buffer's device address on the current device, looked up once per
+// device (host code only holds a stand-in for the symbol, never its address).
 static ssd_status noalloc_scratch(void** out) {
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kNoallocMaxDevices) return SSD_ERR_CUDA;
@@ -477,8 +477,6 @@ static ssd_status noalloc_scratch(void** out) {
   if (!g_noalloc_ptr[dev]) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return SSD_ERR_CUDA;
-    if (cudaMemset(p, 0, SSD_NOALLOC_MAX_WORKSPACE) != cudaSuccess) return SSD_ERR_CUDA;
-    if (cudaDeviceSynchronize() != cudaSuccess) return SSD_ERR_CUDA;
     g_noalloc_ptr[dev] = p;
   }
   *out = g_noalloc_ptr[dev];
@@ -498,6 +496,14 @@ extern "C" ssd_status ssd_verify_noalloc(const void* target_logits, const void* 
   if (B > 0) {
     const ssd_status s = noalloc_scratch(&scratch);
     if (s != SSD_OK) return s;
+    // Every shape lays its counters, decision words, epoch and error word out
+    // at its own offsets, and a timed-out call may leave counters non-zero.
+    // Zeroing this call's control block first, on the call's stream, makes
+    // each call independent of the shape and the fate of the one before.
+    const WsLayout wl = ws_layout(B, K, V, dtype);
+    if (cudaMemsetAsync(static_cast<char*>(scratch) + wl.rflag, 0, wl.total - wl.rflag,
+                        static_cast<cudaStream_t>(stream)) != cudaSuccess)
+      return SSD_ERR_CUDA;
   }
   return ssd_verify(target_logits, draft_logits, draft_next, dtype, B, K, V, draft_tokens, uniforms, T, F, alpha,
                     fanout_mode, C, budget, n_accepted, bonus, out_tokens, accept_prob, residual_mass, cache, status,
