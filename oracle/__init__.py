@@ -45,11 +45,11 @@ def lib():
             [C.c_int] * 5 + [vp, vp, vp, i32p, f32p, C.c_double, i32p, C.c_double, i32p, C.c_uint64,
                              i32p, C.c_int, C.c_int,
                              i32p, i32p, i32p, f64p, f64p, f64p, f64p, f64p, f64p, i32p, i32p,
-                             u8p, i32p, i32p, i32p, f64p, f64p, f64p])
+                             u8p, i32p, i32p, i32p, f64p, f64p, f64p, i32p, i32p])
         L.ssdo_verify_batch.restype = C.c_int
         L.ssdo_reweight_batch.argtypes = (
             [C.c_int] * 5 + [vp, C.c_double, i32p, C.c_double, f32p, i32p, C.c_int, C.c_int,
-                             i32p, i32p, f64p, f64p, f64p, i32p, f64p, i32p])
+                             i32p, i32p, f64p, f64p, f64p, i32p, f64p, i32p, i32p, i32p])
         L.ssdo_reweight_batch.restype = C.c_int
         L.ssdo_overlap.argtypes = [C.c_int, vp, vp, C.c_int, C.c_double]
         L.ssdo_overlap.restype = C.c_double
@@ -152,7 +152,7 @@ def verify(target, draft, tokens, uniforms, T, F=None, C_coef=1.0, budget=0, dra
         offsets=np.zeros((n, K + 2), np.int32), cache_tokens=np.zeros((n, max(budget, 1)), np.int32),
         hit=np.zeros(n, np.uint8), slot=np.zeros(n, np.int32), next_tokens=np.zeros((n, K), np.int32),
         status=np.zeros(n, np.int32), accept_margin=np.zeros(n), bonus_margin=np.zeros(n),
-        p_hit=np.zeros(n))
+        p_hit=np.zeros(n), bonus_lo=np.zeros(n, np.int32), bonus_hi=np.zeros(n, np.int32))
     rc = lib().ssdo_verify_batch(
         _dtype_code(target), B, K, V, budget, _vp(target), _vp(draft), _vp(draft_next),
         _p(tokens, C.c_int32), _p(uniforms, C.c_float), float(T), _p(F, C.c_int32), float(C_coef),
@@ -165,7 +165,8 @@ def verify(target, draft, tokens, uniforms, T, F=None, C_coef=1.0, budget=0, dra
         _p(out["cache_tokens"], C.c_int32) if F is not None else None,
         _p(out["hit"], C.c_uint8), _p(out["slot"], C.c_int32), _p(out["next_tokens"], C.c_int32),
         _p(out["status"], C.c_int32), _p(out["accept_margin"], C.c_double),
-        _p(out["bonus_margin"], C.c_double), _p(out["p_hit"], C.c_double) if want_phit else None)
+        _p(out["bonus_margin"], C.c_double), _p(out["p_hit"], C.c_double) if want_phit else None,
+        _p(out["bonus_lo"], C.c_int32), _p(out["bonus_hi"], C.c_int32))
     if rc != 0:
         raise ValueError("oracle verify rejected its arguments")
     if F is None:
@@ -189,17 +190,21 @@ def reweight(draft, T, F, C_coef, budget, u_draft=None, rows=None, n_threads=Non
     out = dict(topf_tokens=np.full((n, max(budget, 1)), -2, np.int32),
                offsets=np.zeros((n, K + 2), np.int32), Z=np.zeros((n, K)), QS=np.zeros((n, K)),
                q_lse=np.zeros((n, K)), tokens=np.zeros((n, K), np.int32) if u_draft is not None else None,
-               margin=np.zeros(n), status=np.zeros(n, np.int32))
+               margin=np.zeros(n), status=np.zeros(n, np.int32),
+               tok_lo=np.zeros((n, K), np.int32), tok_hi=np.zeros((n, K), np.int32))
     rc = lib().ssdo_reweight_batch(
         _dtype_code(draft), B, K, V, budget, _vp(draft), float(T), _p(F, C.c_int32), float(C_coef),
         _p(u_draft, C.c_float), _p(rows_arr, C.c_int32), n, n_threads or n_threads_default(),
         _p(out["topf_tokens"], C.c_int32), _p(out["offsets"], C.c_int32), _p(out["Z"], C.c_double),
         _p(out["QS"], C.c_double), _p(out["q_lse"], C.c_double), _p(out["tokens"], C.c_int32),
-        _p(out["margin"], C.c_double), _p(out["status"], C.c_int32))
+        _p(out["margin"], C.c_double), _p(out["status"], C.c_int32),
+        _p(out["tok_lo"], C.c_int32) if u_draft is not None else None,
+        _p(out["tok_hi"], C.c_int32) if u_draft is not None else None)
     if rc != 0:
         raise ValueError("oracle reweight rejected its arguments")
     if u_draft is None:
-        out.pop("tokens")
+        for k in ("tokens", "tok_lo", "tok_hi"):
+            out.pop(k)
     return out
 
 

@@ -247,10 +247,16 @@ static double saguaro_row(const double* q, int V, const int32_t* S, int F, doubl
 
 /* Inverse-CDF draw: the smallest v whose running sum of r exceeds u * R, in
  * vocabulary-index order (reading).  If rounding leaves no such v, the last v
- * with r(v) > 0.  *margin = distance of u*R to the nearer CDF step, over R. */
-static int inverse_cdf(const double* r, int V, double R, double u, double* margin) {
+ * with r(v) > 0.  *margin = distance of u*R to the nearer CDF step, over R.
+ * Near-tie window (reading of the 1e-5 decision tolerance): a draw made in
+ * another precision may land anywhere whose CDF interval [c(v-1), c(v)) meets
+ * [u R - 1e-5 R, u R + 1e-5 R]; *wlo and *whi are the lowest and highest
+ * such v among the tokens with r(v) > 0. */
+static int inverse_cdf(const double* r, int V, double R, double u, double* margin, int32_t* wlo,
+                       int32_t* whi) {
   double t = u * R, c = 0.0, prev = 0.0;
-  int last_pos = -1;
+  int last_pos = -1, drawn = -1;
+  *margin = 0.0;
   for (int v = 0; v < V; ++v) {
     prev = c;
     c += r[v];
@@ -258,11 +264,27 @@ static int inverse_cdf(const double* r, int V, double R, double u, double* margi
     if (c > t) {
       double m1 = t - prev, m2 = c - t;
       *margin = (m1 < m2 ? m1 : m2) / R;
-      return v;
+      drawn = v;
+      break;
     }
   }
-  *margin = 0.0;
-  return last_pos < 0 ? V - 1 : last_pos;
+  if (drawn < 0) drawn = last_pos < 0 ? V - 1 : last_pos;
+  const double lo_t = t - SSDO_NEAR_TIE * R, hi_t = t + SSDO_NEAR_TIE * R;
+  int lo = -1, hi = -1;
+  c = 0.0;
+  for (int v = 0; v < V; ++v) {
+    prev = c;
+    c += r[v];
+    if (!(r[v] > 0.0)) continue;
+    if (lo < 0 && c > lo_t) lo = v;
+    if (prev <= hi_t) hi = v;
+  }
+  if (lo < 0 || hi < 0) lo = hi = drawn;
+  if (drawn < lo) lo = drawn;
+  if (drawn > hi) hi = drawn;
+  *wlo = lo;
+  *whi = hi;
+  return drawn;
 }
 
 /* ------------------------------------------------------------------------- */
@@ -287,6 +309,7 @@ typedef struct {
   int32_t* offsets; int32_t* cache_tokens;
   uint8_t* hit; int32_t* slot; int32_t* next_tokens;
   int32_t* status; double* accept_margin; double* bonus_margin; double* p_hit;
+  int32_t* bonus_lo; int32_t* bonus_hi;
 } verify_job;
 
 static void verify_row(const verify_job* J, int i) {
@@ -358,6 +381,8 @@ static void verify_row(const verify_job* J, int i) {
     if (J->accept_margin) J->accept_margin[i] = INFINITY;
     if (J->bonus_margin) J->bonus_margin[i] = INFINITY;
     if (J->p_hit) J->p_hit[i] = NAN;
+    if (J->bonus_lo) J->bonus_lo[i] = -1;
+    if (J->bonus_hi) J->bonus_hi[i] = -1;
     goto done;
   }
 
@@ -373,6 +398,7 @@ static void verify_row(const verify_job* J, int i) {
     }
     double* a = malloc(sizeof(double) * (size_t)K);
     int kstar = K, bon = -1;
+    int32_t blo = -1, bhi = -1;
     double R = 1.0, amarg = INFINITY, bmarg = INFINITY, phit = NAN;
 
     if (J->T == 0.0) {
@@ -394,6 +420,7 @@ static void verify_row(const verify_job* J, int i) {
       if (J->p_lse)
         for (int j = 0; j <= K; ++j) J->p_lse[(size_t)i * (K + 1) + j] = lp[j][argmax_row(lp[j], V)];
       bon = argmax_row(lp[kstar], V);
+      blo = bhi = bon;
       R = 1.0;
     } else {
       double** p = malloc(sizeof(double*) * (size_t)(K + 1));
@@ -456,7 +483,7 @@ static void verify_row(const verify_job* J, int i) {
         R = 0.0;
         for (int v = 0; v < V; ++v) { r[v] = p[K][v]; R += r[v]; }
       }
-      bon = inverse_cdf(r, V, R, uK, &bmarg);
+      bon = inverse_cdf(r, V, R, uK, &bmarg, &blo, &bhi);
 
       if (J->p_hit && F) {
         /* Diagnostic: probability that the outcome (k*, bonus) lands in the
@@ -515,6 +542,8 @@ static void verify_row(const verify_job* J, int i) {
     if (J->accept_margin) J->accept_margin[i] = amarg;
     if (J->bonus_margin) J->bonus_margin[i] = bmarg;
     if (J->p_hit) J->p_hit[i] = phit;
+    if (J->bonus_lo) J->bonus_lo[i] = blo;
+    if (J->bonus_hi) J->bonus_hi[i] = bhi;
     for (int k = 0; k <= K; ++k) free(S[k]);
     free(S); free(a);
   }
@@ -561,7 +590,8 @@ int ssdo_verify_batch(int dtype, int B, int K, int V, int budget,
                       double* Z, double* QS, double* q_lse, double* p_lse,
                       int32_t* offsets, int32_t* cache_tokens,
                       uint8_t* hit, int32_t* slot, int32_t* next_tokens,
-                      int32_t* status, double* accept_margin, double* bonus_margin, double* p_hit) {
+                      int32_t* status, double* accept_margin, double* bonus_margin, double* p_hit,
+                      int32_t* bonus_lo, int32_t* bonus_hi) {
   if (B < 0 || K < 1 || V < 1 || !(T >= 0.0) || (F && !(C > 0.0 && C <= 1.0))) return -1;
   if (dtype != SSDO_DTYPE_FP32 && dtype != SSDO_DTYPE_BF16) return -1;
   if (F && (budget < 0 || budget > V)) return -1;
@@ -569,7 +599,7 @@ int ssdo_verify_batch(int dtype, int B, int K, int V, int budget,
                   payload, fallback_seed, rows, rows ? n_rows : B, n_threads,
                   n_accepted, bonus, out_tokens, accept_prob, residual_mass, Z, QS, q_lse, p_lse,
                   offsets, cache_tokens, hit, slot, next_tokens, status, accept_margin,
-                  bonus_margin, p_hit};
+                  bonus_margin, p_hit, bonus_lo, bonus_hi};
   run_rows(&J, J.n_rows, n_threads, verify_row_thunk);
   return 0;
 }
@@ -585,6 +615,7 @@ typedef struct {
   const int32_t* rows; int n_rows;
   int32_t* topf_tokens; int32_t* offsets; double* Z; double* QS; double* q_lse;
   int32_t* tokens_out; double* margin; int32_t* status;
+  int32_t* tok_lo; int32_t* tok_hi;  /* [n, K] near-tie windows of the draws, or NULL */
 } reweight_job;
 
 static void reweight_row(const void* jp, int i) {
@@ -620,6 +651,7 @@ static void reweight_row(const void* jp, int i) {
       J->Z[o] = NAN; J->QS[o] = NAN; J->q_lse[o] = NAN;
       if (!(st & SSDO_ROW_BAD_PLAN)) for (int s = 0; s < F[j]; ++s) seg[s] = -1;
       if (J->tokens_out) J->tokens_out[o] = -1;
+      if (J->tok_lo) { J->tok_lo[o] = -1; J->tok_hi[o] = -1; }
       continue;
     }
     topf_row(l, V, F[j], seg);
@@ -629,6 +661,7 @@ static void reweight_row(const void* jp, int i) {
       for (int s = 0; s < F[j]; ++s) if (seg[s] == am) qs = 1.0;
       J->Z[o] = 1.0; J->QS[o] = qs; J->q_lse[o] = l[am];
       if (J->tokens_out) J->tokens_out[o] = am;
+      if (J->tok_lo) { J->tok_lo[o] = am; J->tok_hi[o] = am; }
       continue;
     }
     J->q_lse[o] = softmax_row(l, V, J->T, q);
@@ -637,8 +670,11 @@ static void reweight_row(const void* jp, int i) {
     J->QS[o] = QSj;
     if (J->tokens_out) {
       double tot = 0.0, mg;
+      int32_t wl, wh;
       for (int v = 0; v < V; ++v) tot += qp[v];
-      J->tokens_out[o] = inverse_cdf(qp, V, tot, (double)J->u_draft[(size_t)b * (size_t)K + (size_t)j], &mg);
+      J->tokens_out[o] = inverse_cdf(qp, V, tot, (double)J->u_draft[(size_t)b * (size_t)K + (size_t)j], &mg,
+                                     &wl, &wh);
+      if (J->tok_lo) { J->tok_lo[o] = wl; J->tok_hi[o] = wh; }
       if (mg < worst) worst = mg;
     }
   }
@@ -652,13 +688,14 @@ int ssdo_reweight_batch(int dtype, int B, int K, int V, int budget, const void* 
                         const int32_t* F, double C, const float* u_draft,
                         const int32_t* rows, int n_rows, int n_threads,
                         int32_t* topf_tokens, int32_t* offsets, double* Z, double* QS, double* q_lse,
-                        int32_t* tokens_out, double* margin, int32_t* status) {
+                        int32_t* tokens_out, double* margin, int32_t* status, int32_t* tok_lo,
+                        int32_t* tok_hi) {
   if (B < 0 || K < 1 || V < 1 || !(T >= 0.0) || !(C > 0.0 && C <= 1.0) || !F) return -1;
   if (budget < 0 || budget > V) return -1;
   if (dtype != SSDO_DTYPE_FP32 && dtype != SSDO_DTYPE_BF16) return -1;
   if (tokens_out && !u_draft) return -1;
   reweight_job J = {dtype, B, K, V, budget, draft, T, F, C, u_draft, rows, rows ? n_rows : B,
-                    topf_tokens, offsets, Z, QS, q_lse, tokens_out, margin, status};
+                    topf_tokens, offsets, Z, QS, q_lse, tokens_out, margin, status, tok_lo, tok_hi};
   run_rows(&J, J.n_rows, n_threads, reweight_row);
   return 0;
 }

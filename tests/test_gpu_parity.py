@@ -99,7 +99,7 @@ FULL = ["zipf_b16_k5_v32000_bf16", "zipf_b64_k6_v128256_bf16", "zipf_b256_k8_v15
 def test_verify_full_size_sampled(name):
     w = W[name]
     rng = np.random.default_rng(99)
-    rows = np.sort(rng.choice(w.B, size=min(w.B, 12), replace=False)).astype(np.int32)
+    rows = np.sort(rng.choice(w.B, size=min(w.B, 24), replace=False)).astype(np.int32)
     case = Case(w, check_rows=rows)
     gpu = case.run_gpu()
     orc = case.run_oracle()
@@ -236,9 +236,15 @@ def test_saguaro_reweight_and_draft_draw(name, T):
         np.testing.assert_array_equal(tg[b, :n_keys[b]], o["topf_tokens"][b, :n_keys[b]])
     assert np.max(np.abs(r.Z.cpu().numpy() - o["Z"])) < PROB_ATOL
     ql = r.q_lse.cpu().numpy().astype(np.float64)
-    assert np.max(np.abs(ql - o["q_lse"]) / np.maximum(1.0, np.abs(o["q_lse"]))) < LSE_RTOL * 4
+    lse_err = np.max(np.abs(ql - o["q_lse"]) / np.maximum(1.0, np.abs(o["q_lse"])))
+    print(f"q_lse error relative to max(1, |lse|): {lse_err:.3g}")
+    assert lse_err < LSE_RTOL
+    # every draft token is bit-exact, or inside the oracle's near-tie window
+    # of its draw when that draw's margin is below 1e-5
+    dg = r.draft_tokens.cpu().numpy()
+    assert np.all((o["tok_lo"] <= dg) & (dg <= o["tok_hi"]))
     near = (o["status"] & oracle.ROW_NEAR_TIE) != 0
-    np.testing.assert_array_equal(r.draft_tokens.cpu().numpy()[~near], o["tokens"][~near])
+    np.testing.assert_array_equal(dg[~near], o["tokens"][~near])
 
 
 def test_unfused_pipeline_equals_fused():
@@ -261,6 +267,9 @@ def test_unfused_pipeline_equals_fused():
     hit, slot, nxt = ssd.ssd_cache_lookup(offs, toks, ver.n_accepted, ver.bonus, V,
                                           fallback_seed=w.fallback_seed)
     torch.cuda.synchronize()
+    orc = case.run_oracle()
+    np.testing.assert_array_equal(offs.cpu().numpy(), orc["offsets"])
+    np.testing.assert_array_equal(toks.cpu().numpy(), orc["cache_tokens"])
     np.testing.assert_array_equal(offs.cpu().numpy(), fused["cache_offsets"])
     np.testing.assert_array_equal(toks.cpu().numpy(), fused["cache_tokens"])
     for a, bname in ((ver.n_accepted, "n_accepted"), (ver.bonus, "bonus"), (hit, "hit"), (slot, "slot"),

@@ -557,3 +557,122 @@ def test_bonus_uses_the_last_uniform_whatever_k_star():
     assert out["n_accepted"][0] == 0 and out["accept_prob"][0, 0] == 0.0
     assert out["residual_mass"][0] == 1.0
     assert out["bonus"][0] == 1
+
+
+# ---------------------------------------------------------------------------
+# The decision margins and near-tie windows (the 1e-5 decision tolerance):
+# exact on the dyadic cases above, where every CDF step and every a_j is a
+# power of two, and by brute force over the CDF intervals on small rows.
+# ---------------------------------------------------------------------------
+def test_decision_margins_exact_at_dyadic_boundaries():
+    p = [[0, 0, 0, 0], [0, 0, 0, 0]]
+    q = [[0, 0, NEG, NEG]]
+    u3 = float(np.float32(0.3))
+    # u_0 = a_0 = 1/2: rejected with margin 0.  r = (0, 0, 1/4, 1/4), R = 1/2,
+    # t = u_K R with u_K = 0.3 falls inside token 2's interval [0, 1/4): its
+    # distance to the step at 1/4, over R, is 1/2 - u_K.
+    at = _one_row(p, q, [0], [0.5, 0.3])
+    assert at["accept_margin"][0] == 0.0
+    assert at["bonus_margin"][0] == (0.25 - u3 * 0.5) / 0.5
+    assert at["bonus_lo"][0] == 2 and at["bonus_hi"][0] == 2
+    # u_0 one grid step below a_0: accepted with margin 2^-24, then the full
+    # acceptance draw from p_1 = (1/4, 1/4, 1/4, 1/4): t = 0.3 lies between the
+    # steps 1/4 and 1/2, margin min(0.3 - 1/4, 1/2 - 0.3) / 1.
+    below = _one_row(p, q, [0], [0.5 - 2.0 ** -24, 0.3])
+    assert below["n_accepted"][0] == 1 and below["bonus"][0] == 1
+    assert below["accept_margin"][0] == 2.0 ** -24
+    assert below["bonus_margin"][0] == min(u3 - 0.25, 0.5 - u3)
+    assert below["bonus_lo"][0] == 1 and below["bonus_hi"][0] == 1
+    # t exactly on the step at 1/4 between tokens 2 and 3: margin 0, and the
+    # window holds both neighbours; one grid step below it, margin 2^-25 / R.
+    on = _one_row(p, q, [0], [0.5, 0.5])
+    assert on["bonus"][0] == 3 and on["bonus_margin"][0] == 0.0
+    assert on["bonus_lo"][0] == 2 and on["bonus_hi"][0] == 3
+    near = _one_row(p, q, [0], [0.5, 0.5 - 2.0 ** -24])
+    assert near["bonus"][0] == 2 and near["bonus_margin"][0] == 2.0 ** -24
+    assert near["bonus_lo"][0] == 2 and near["bonus_hi"][0] == 3
+    # a row that never reaches a tie: its margin is the smallest |u_j - a_j|
+    # over the tests it ran (positions 0..k*), here u_0 = 1/8 vs a_0 = 1/2
+    far = _one_row(p, q, [0], [0.125, 0.3])
+    assert far["accept_margin"][0] == 0.375
+
+
+def _window_brute(r, t, delta):
+    """Tokens with mass whose CDF interval [c(v-1), c(v)) meets [t - delta, t + delta]."""
+    c = np.cumsum(r)
+    prev = c - r
+    hit = (r > 0) & (c > t - delta) & (prev <= t + delta)
+    idx = np.nonzero(hit)[0]
+    return int(idx.min()), int(idx.max())
+
+
+@pytest.mark.parametrize("seed", range(4))
+def test_bonus_window_matches_brute_force(seed):
+    """Full acceptance (q = p, C = 1) makes k* = K, so the bonus is the inverse
+    CDF of p_K at u_K: the oracle's window equals the set of tokens whose CDF
+    interval meets [t - 1e-5, t + 1e-5], found by brute force here, and it
+    always contains the drawn token.  Quantised logits put many tiny steps
+    close together, so the windows are wide."""
+    rng = np.random.default_rng(seed)
+    K, V, n = 2, 64, 200
+    lp = np.round(rng.normal(0, 3, (K + 1, V)) * 2) / 2
+    lp[K, rng.choice(V, 5, replace=False)] = -np.inf
+    lp = lp.astype(np.float32)
+    target = tile_rows(lp, n)
+    draft = tile_rows(lp[:K], n)
+    D = np.zeros((n, K), np.int32)
+    U = np.zeros((n, K + 1), np.float32)
+    U[:, K] = synth.uniforms(seed, n, 1, 0)[:, 0]
+    out = oracle.verify(target, draft, D, U, 1.0, n_threads=1)
+    assert np.all(out["n_accepted"] == K)
+    pK = softmax64(lp[K], 1.0)
+    for i in range(n):
+        t = float(U[i, K]) * pK.sum()
+        lo, hi = _window_brute(pK, t, 1e-5 * pK.sum())
+        assert (out["bonus_lo"][i], out["bonus_hi"][i]) == (lo, hi), i
+        assert lo <= out["bonus"][i] <= hi
+
+
+def test_draft_draw_window_on_a_dyadic_case():
+    """The draft draw d ~ q' shares the inverse CDF: q_0 = (1/4, 1/4, 1/2, 0)
+    with C = 1; u = 1/2 sits exactly on the step after token 1."""
+    with np.errstate(divide="ignore"):
+        lq = np.log(np.array([[[1.0, 1.0, 2.0, 0.0]]], np.float64)).astype(np.float32)
+    F = np.array([[0, 0]], np.int32)
+    r = oracle.reweight(lq, 1.0, F, 1.0, 0, u_draft=np.array([[0.5]], np.float32), n_threads=1)
+    assert r["tokens"][0, 0] == 2
+    assert r["tok_lo"][0, 0] == 1 and r["tok_hi"][0, 0] == 2
+    r = oracle.reweight(lq, 1.0, F, 1.0, 0, u_draft=np.array([[0.75]], np.float32), n_threads=1)
+    assert r["tokens"][0, 0] == 2 and r["tok_lo"][0, 0] == 2 and r["tok_hi"][0, 0] == 2
+
+
+# ---------------------------------------------------------------------------
+# Log-normalisers: closed forms, and the library log-sum-exp on random rows.
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("T", [1.0, 0.7, 2.5])
+def test_log_normalisers_closed_forms(T):
+    """A row of V equal logits L has lse = L / T + ln V; a row with n zeros
+    and the rest -inf has lse = ln n (any T).  Checked for the target rows
+    (p_lse) and the draft rows (q_lse)."""
+    K, V = 2, 24
+    L = np.float32(1.75)
+    lp = np.full((K + 1, V), L, np.float32)
+    lq = np.full((K, V), NEG, np.float32)
+    lq[0, :5] = 0.0
+    lq[1, :16] = 0.0
+    out = oracle.verify(lp[None], lq[None], np.zeros((1, K), np.int32), np.zeros((1, K + 1), np.float32), T,
+                        n_threads=1)
+    np.testing.assert_allclose(out["p_lse"][0], float(L) / T + np.log(V), rtol=0, atol=1e-14)
+    np.testing.assert_allclose(out["q_lse"][0], [np.log(5.0), np.log(16.0)], rtol=0, atol=1e-14)
+
+
+def test_log_normalisers_match_library_logsumexp():
+    from scipy.special import logsumexp
+    rng = np.random.default_rng(8)
+    K, V, T = 3, 1000, 0.8
+    lp = rng.normal(0, 4, (2, K + 1, V)).astype(np.float32)
+    lq = rng.normal(0, 4, (2, K, V)).astype(np.float32)
+    lq[1, 0, :900] = -np.inf
+    out = oracle.verify(lp, lq, np.zeros((2, K), np.int32), np.zeros((2, K + 1), np.float32), T, n_threads=1)
+    np.testing.assert_allclose(out["p_lse"], logsumexp(lp.astype(np.float64) / T, axis=2), rtol=1e-14, atol=0)
+    np.testing.assert_allclose(out["q_lse"], logsumexp(lq.astype(np.float64) / T, axis=2), rtol=1e-14, atol=0)
