@@ -105,6 +105,60 @@ ssd_status ssd_fanout_plan(const float* alpha, int B, int K, int budget, int mod
                            int32_t* F, void* stream);
 
 /*
+ * ssd_fanout_plan_power -- the power-law fan-out ([ZH] section 2, challenge
+ * 1: the split follows the power law of the acceptance and is the solution of
+ * a constrained optimisation; [NL] section 3A: a geometric series).  Reading:
+ * when the hit rate of an outcome given F bonus guesses follows a power-law
+ * curve 1 - c F^-beta, the budget-constrained optimum of the expected hit
+ * rate puts F_k proportional to P(k)^gamma, gamma = 1 / (1 + beta): still
+ * geometric in k, with ratio alpha^gamma.  gamma = gamma_eighths / 8,
+ * gamma_eighths in 1..8 (8 is exactly ssd_fanout_plan's geometric plan).
+ * alpha^gamma and (1 - alpha)^gamma are formed from three correctly rounded
+ * square roots and gamma_eighths - 1 products; weights w_k = a^k c (k < K),
+ * w_K = a^K; quotas budget * w_k / (w_0 + ... + w_K); largest remainder, ties
+ * to the smaller k.  fp64, every operation rounded on its own.
+ *   alpha [B] fp32 in [0, 1] (outside: F = 0 with -1 in F[b,0]); F [B, K+1]
+ *   int32 out.  0 <= budget <= SSD_MAX_BUDGET.  Feed F to ssd_verify.
+ */
+ssd_status ssd_fanout_plan_power(const float* alpha, int B, int K, int budget, int gamma_eighths,
+                                 int32_t* F, void* stream);
+
+/*
+ * ssd_alpha_update -- per-row acceptance estimate from history, the input of
+ * the fan-out plans ([ZH] section 2, challenge 1: the split follows the
+ * acceptance).  Reading: a_j is the expected acceptance of position j given
+ * the drafts, so one step's estimate of the per-token acceptance is the mean
+ * of accept_prob[b, 0..K-1], and alpha follows it by exponential smoothing:
+ * alpha_out[b] = (1 - lambda) alpha[b] + lambda mean_j a_j (fp64, rounded
+ * to fp32).  Rows with an SSD_ROW_INVALID bit, or a NaN a_j, keep alpha[b].
+ *   alpha [B], accept_prob [B, K] (as ssd_verify writes it), status [B] in;
+ *   alpha_out [B] out (may equal alpha).  0 <= lambda <= 1.
+ */
+ssd_status ssd_alpha_update(const float* alpha, const float* accept_prob, const int32_t* status, int B,
+                            int K, double lambda, float* alpha_out, void* stream);
+
+/*
+ * ssd_fallback_bstar -- the fallback speculator by batch size ([ZH] section
+ * 2, challenge 3; [NL] section 3C: a slow high-quality fallback for small
+ * batches, a fast low-quality one -- n-gram or random tokens -- for large
+ * ones, switching at a critical batch size b*).  HOST function, no device
+ * work.  Reading: each row hits the cache with probability h; when any row
+ * of a batch of b misses, the whole batch waits for the fallback, so a round
+ * lasts L_target + (1 - h^b) L_fallback.  A hit, or a miss served by the
+ * primary speculator, yields E_p = sum_{i=0..K} alpha^i tokens (expected
+ * accepted drafts plus the bonus); a miss served by the fast one yields
+ * E_fast.  The fast fallback is chosen for b when its expected tokens per
+ * unit time are strictly higher.
+ *   h: per-row hit probability (e.g. the mean of ssd_cache.hit); alpha:
+ *   per-token acceptance; latencies in any one unit; choice: NULL or a HOST
+ *   array of b_max bytes, choice[b-1] = 1 when batch size b takes the fast
+ *   fallback.  Returns b* (the smallest such b), b_max + 1 when none does,
+ *   -1 for arguments out of range.
+ */
+int ssd_fallback_bstar(double h, double alpha, int K, double L_target, double L_primary, double L_fast,
+                       double E_fast, int b_max, uint8_t* choice);
+
+/*
  * ssd_saguaro_reweight -- draft side ([ZH] section 2, challenge 2; [NL]
  * section 3B): for every (b, j < K), the top-F[b,j] tokens S_j of the draft
  * distribution q_j (by raw logit, ties to the lower id), Q_S = sum_{S_j} q_j,
@@ -193,6 +247,31 @@ ssd_status ssd_verify_noalloc(const void* target_logits, const void* draft_logit
                               int32_t* n_accepted, int32_t* bonus, int32_t* out_tokens,
                               float* accept_prob, float* residual_mass, const ssd_cache* cache,
                               int32_t* status, void* stream);
+
+/*
+ * ssd_prespeculate -- pre-speculation of the cache payload ([ZH] section 2,
+ * basic flow step 3: for each predicted verification outcome the draft
+ * generates the following tokens in advance and stores them in the
+ * speculation cache; [NL] section 2, "speculation cache").  For every cache
+ * key s of row b the caller's draft model has produced logits for the K
+ * positions after that key; this draws the K draft tokens of the key with
+ * Saguaro sampling of the NEXT round ([ZH] challenge 2): d_i ~ q'_i, the
+ * top-F_next[.,i] tokens of q_i down-weighted by C and renormalised, by
+ * inverse CDF in token order with the caller's uniforms -- exactly
+ * ssd_saguaro_reweight's draw on B * n_keys rows.
+ *   key_logits [B, n_keys, K, V] (bf16 or fp32, 16-byte aligned);
+ *   F_next [B * n_keys, K+1] the next round's plan per key (zeros with
+ *   next_budget = 0 for plain sampling from q); 0 < C <= 1;
+ *   uniforms [B, n_keys, K] in [0, 1); payload [B, n_keys, K] int32 out (the
+ *   ssd_cache.payload layout when n_keys = budget); status [B * n_keys] out
+ *   (SSD_ROW_* bits; an invalid key row gets -1 tokens).
+ *   workspace: ssd_workspace_bytes(B * n_keys, K, V, dtype) bytes.
+ *   T = 0 draws the argmax of each q_i.
+ */
+ssd_status ssd_prespeculate(const void* key_logits, int dtype, int B, int n_keys, int K, int V, float T,
+                            const int32_t* F_next, float C, int next_budget, const float* uniforms,
+                            int32_t* payload, int32_t* status, void* workspace, size_t ws_bytes,
+                            void* stream);
 
 /*
  * ssd_cache_build -- pack per-outcome guess lists into the cache layout

@@ -39,6 +39,13 @@ def lib():
         L.ssdo_fallback_token.restype = C.c_int32
         L.ssdo_fanout_plan.argtypes = [C.c_double, C.c_int, C.c_int, C.c_int, i32p]
         L.ssdo_fanout_plan.restype = C.c_int
+        L.ssdo_fanout_plan_power.argtypes = [C.c_double, C.c_int, C.c_int, C.c_int, i32p]
+        L.ssdo_fanout_plan_power.restype = C.c_int
+        L.ssdo_alpha_update.argtypes = [C.c_int, C.c_int, f32p, f32p, i32p, C.c_double, f32p]
+        L.ssdo_alpha_update.restype = None
+        L.ssdo_fallback_bstar.argtypes = [C.c_double, C.c_double, C.c_int, C.c_double, C.c_double, C.c_double,
+                                          C.c_double, C.c_int, u8p]
+        L.ssdo_fallback_bstar.restype = C.c_int
         L.ssdo_topf.argtypes = [f64p, C.c_int, C.c_int, i32p]
         L.ssdo_topf.restype = C.c_int
         L.ssdo_verify_batch.argtypes = (
@@ -106,6 +113,38 @@ def fanout_plan(alpha, K, budget, mode=0):
 def fanout_plan_batch(alpha, K, budget, mode=0):
     alpha = np.asarray(alpha, dtype=np.float32)
     return np.stack([fanout_plan(float(a), K, budget, mode) for a in alpha])
+
+
+def fanout_plan_power(alpha, K, budget, q):
+    """Power-law plan, gamma = q / 8 (q = 8: the geometric plan)."""
+    F = np.zeros(K + 1, dtype=np.int32)
+    if lib().ssdo_fanout_plan_power(float(alpha), K, budget, int(q), _p(F, C.c_int32)) != 0:
+        raise ValueError("bad fan-out arguments")
+    return F
+
+
+def fanout_plan_power_batch(alpha, K, budget, q):
+    alpha = np.asarray(alpha, dtype=np.float32)
+    return np.stack([fanout_plan_power(float(a), K, budget, q) for a in alpha])
+
+
+def alpha_update(alpha, accept_prob, status, lam):
+    alpha = np.ascontiguousarray(alpha, dtype=np.float32)
+    ap = np.ascontiguousarray(accept_prob, dtype=np.float32)
+    st = np.ascontiguousarray(status, dtype=np.int32)
+    B, K = ap.shape
+    out = np.zeros(B, np.float32)
+    lib().ssdo_alpha_update(B, K, _p(alpha, C.c_float), _p(ap, C.c_float), _p(st, C.c_int32), float(lam),
+                            _p(out, C.c_float))
+    return out
+
+
+def fallback_bstar(h, alpha, K, L_target, L_primary, L_fast, E_fast, b_max):
+    """(b*, choice[b_max]) of the batch-size fallback policy."""
+    choice = np.zeros(b_max, np.uint8)
+    bs = lib().ssdo_fallback_bstar(float(h), float(alpha), int(K), float(L_target), float(L_primary),
+                                   float(L_fast), float(E_fast), int(b_max), _p(choice, C.c_uint8))
+    return int(bs), choice
 
 
 def topf(logits, F):

@@ -172,6 +172,119 @@ int ssdo_fanout_plan(double alpha, int K, int budget, int mode, int32_t* F) {
   return 0;
 }
 
+/* Power-law fan-out ([ZH] section 2, challenge 1: the acceptance follows a
+ * power law and the split is a constrained optimisation; [NL] section 3A: the
+ * optimal split is a geometric series).  Reading: if the hit rate of an
+ * outcome given F guesses follows a power-law curve 1 - c F^-beta, the
+ * budget-constrained optimum of sum_k P(k) h(F_k) puts F_k proportional to
+ * P(k)^gamma with gamma = 1 / (1 + beta) -- still a geometric series in k,
+ * of ratio alpha^gamma.  gamma = q / 8, q = 1..8.  alpha^gamma and
+ * (1 - alpha)^gamma are formed from three square roots (the eighth root) and
+ * q - 1 products, so every evaluation of the plan gives the same numbers.
+ * Weights w_k = a^k c (k < K), w_K = a^K with a = alpha^gamma, c =
+ * (1 - alpha)^gamma; quotas budget * w_k / W, W = w_0 + ... + w_K in that
+ * order; largest remainder as for the geometric plan.  q = 8 is the
+ * geometric plan itself. */
+static double eighth_power(double x, int q) {
+  double r = sqrt(sqrt(sqrt(x)));
+  double y = r;
+  for (int i = 1; i < q; ++i) y = y * r;
+  return y;
+}
+
+int ssdo_fanout_plan_power(double alpha, int K, int budget, int q, int32_t* F) {
+  if (K < 1 || budget < 0 || q < 1 || q > 8 || !(alpha >= 0.0 && alpha <= 1.0)) return -1;
+  if (q == 8) return ssdo_fanout_plan(alpha, K, budget, 0, F);
+  double a = eighth_power(alpha, q), c = eighth_power(1.0 - alpha, q);
+  double* w = malloc(sizeof(double) * (size_t)(K + 1));
+  double* frac = malloc(sizeof(double) * (size_t)(K + 1));
+  int* taken = calloc((size_t)(K + 1), sizeof(int));
+  double run = 1.0, W = 0.0;
+  for (int k = 0; k < K; ++k) {
+    w[k] = run * c;
+    run = run * a;
+  }
+  w[K] = run;
+  for (int k = 0; k <= K; ++k) W = W + w[k];
+  long assigned = 0;
+  for (int k = 0; k <= K; ++k) {
+    double quota = (double)budget * w[k] / W;
+    double fl = floor(quota);
+    F[k] = (int32_t)fl;
+    frac[k] = quota - fl;
+    assigned += F[k];
+  }
+  long rem = (long)budget - assigned;
+  while (rem > 0) {
+    int best = -1;
+    for (int k = 0; k <= K; ++k)
+      if (!taken[k] && (best < 0 || frac[k] > frac[best])) best = k;
+    if (best < 0) {
+      memset(taken, 0, sizeof(int) * (size_t)(K + 1));
+      continue;
+    }
+    taken[best] = 1;
+    F[best] += 1;
+    --rem;
+  }
+  free(w); free(frac); free(taken);
+  return 0;
+}
+
+/* Per-row acceptance estimate from history ([ZH] section 2, challenge 1:
+ * the fan-out follows the acceptance, which differs between requests).
+ * Reading: the expected acceptance of position j given the drafts is a_j,
+ * so the step's estimate of the per-token acceptance is the mean of a_j over
+ * the K positions, and the row's alpha follows it by exponential smoothing:
+ * alpha' = (1 - lambda) alpha + lambda mean_j a_j, in double, rounded to
+ * float.  Rows flagged invalid, or with a NaN a_j, keep their alpha. */
+void ssdo_alpha_update(int B, int K, const float* alpha, const float* accept_prob, const int32_t* status,
+                       double lambda, float* alpha_out) {
+  for (int b = 0; b < B; ++b) {
+    int ok = !(status[b] & SSDO_ROW_INVALID);
+    double s = 0.0;
+    for (int j = 0; j < K; ++j) {
+      double a = (double)accept_prob[(size_t)b * K + j];
+      if (isnan(a)) ok = 0;
+      s = s + a;
+    }
+    if (!ok) { alpha_out[b] = alpha[b]; continue; }
+    double mean = s / (double)K;
+    alpha_out[b] = (float)((1.0 - lambda) * (double)alpha[b] + lambda * mean);
+  }
+}
+
+/* Fallback speculator by batch size ([ZH] section 2, challenge 3; [NL]
+ * section 3C: a slow high-quality fallback for small batches, a fast
+ * low-quality one (random tokens) for large ones, switching at a critical
+ * batch size b*).  Reading: a row hits the cache with probability h,
+ * independently; on any miss in the batch the whole batch waits for the
+ * fallback.  A round takes L_target plus, with probability 1 - h^b, the
+ * fallback's latency.  A hit, or a miss with the primary fallback, yields
+ * E_p = sum_{i=0..K} alpha^i tokens (expected accepted drafts plus the
+ * bonus); a miss with the fast fallback yields E_f.  The fast fallback is
+ * chosen when its expected tokens per unit time are strictly higher.
+ * Returns b* = the smallest b in [1, b_max] that chooses the fast fallback,
+ * b_max + 1 when none does; choice[b-1] = 1 for the fast one, 0 otherwise
+ * (choice may be NULL). */
+int ssdo_fallback_bstar(double h, double alpha, int K, double L_target, double L_primary, double L_fast,
+                        double E_fast, int b_max, uint8_t* choice) {
+  double Ep = 0.0, ak = 1.0;
+  for (int i = 0; i <= K; ++i) { Ep = Ep + ak; ak = ak * alpha; }
+  int bstar = b_max + 1;
+  double hb = 1.0;
+  for (int b = 1; b <= b_max; ++b) {
+    hb = hb * h;
+    double miss_any = 1.0 - hb;
+    double thr_primary = Ep / (L_target + miss_any * L_primary);
+    double thr_fast = (h * Ep + (1.0 - h) * E_fast) / (L_target + miss_any * L_fast);
+    int fast = thr_fast > thr_primary;
+    if (choice) choice[b - 1] = (uint8_t)fast;
+    if (fast && bstar > b_max) bstar = b;
+  }
+  return bstar;
+}
+
 /* ------------------------------------------------------------------------- */
 /* Top-F of a logit row: the first F entries of the row sorted by (logit      */
 /* descending, index ascending).  Softmax is monotone for T > 0, so this is   */

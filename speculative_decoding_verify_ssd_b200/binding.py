@@ -82,6 +82,15 @@ def load(build_if_missing: bool = True):
     L.ssd_verify_noalloc.restype = i32
     L.ssd_verify_noalloc.argtypes = [vp, vp, vp, i32, i32, i32, i32, vp, vp, f32, vp, vp, i32, f32, i32, vp, vp,
                                      vp, vp, vp, C.POINTER(_Cache), vp, vp]
+    L.ssd_fanout_plan_power.restype = i32
+    L.ssd_fanout_plan_power.argtypes = [vp, i32, i32, i32, i32, vp, vp]
+    L.ssd_alpha_update.restype = i32
+    L.ssd_alpha_update.argtypes = [vp, vp, vp, i32, i32, C.c_double, vp, vp]
+    L.ssd_fallback_bstar.restype = i32
+    L.ssd_fallback_bstar.argtypes = [C.c_double, C.c_double, i32, C.c_double, C.c_double, C.c_double, C.c_double,
+                                     i32, vp]
+    L.ssd_prespeculate.restype = i32
+    L.ssd_prespeculate.argtypes = [vp, i32, i32, i32, i32, i32, f32, vp, f32, i32, vp, vp, vp, vp, sz, vp]
     L.ssd_cache_build.restype = i32
     L.ssd_cache_build.argtypes = [vp, vp, vp, i32, i32, i32, vp, vp, vp]
     L.ssd_cache_lookup.restype = i32
@@ -198,6 +207,71 @@ def ssd_fanout_plan(alpha: torch.Tensor, K: int, budget: int, mode: int = FANOUT
         _check(load().ssd_fanout_plan(_ptr(alpha), B, K, budget, mode, _ptr(F), _stream(stream)),
                "ssd_fanout_plan")
     return F
+
+
+def ssd_fanout_plan_power(alpha: torch.Tensor, K: int, budget: int, gamma_eighths: int,
+                          F: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Power-law fan-out plan, gamma = gamma_eighths / 8 (see ssd.h)."""
+    B = alpha.shape[0]
+    _need(alpha, "alpha", torch.float32, (B,), alpha.device)
+    if F is None:
+        F = torch.empty((B, K + 1), dtype=torch.int32, device=alpha.device)
+    _need(F, "F", torch.int32, (B, K + 1), alpha.device)
+    with torch.cuda.device(alpha.device):
+        _check(load().ssd_fanout_plan_power(_ptr(alpha), B, K, budget, int(gamma_eighths), _ptr(F),
+                                            _stream(stream)), "ssd_fanout_plan_power")
+    return F
+
+
+def ssd_alpha_update(alpha: torch.Tensor, accept_prob: torch.Tensor, status: torch.Tensor, lam: float,
+                     out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """alpha' = (1 - lam) alpha + lam * mean_j accept_prob[:, j] per valid row."""
+    B, K = accept_prob.shape
+    dev = alpha.device
+    _need(alpha, "alpha", torch.float32, (B,), dev)
+    _need(accept_prob, "accept_prob", torch.float32, (B, K), dev)
+    _need(status, "status", torch.int32, (B,), dev)
+    if out is None:
+        out = torch.empty_like(alpha)
+    with torch.cuda.device(dev):
+        _check(load().ssd_alpha_update(_ptr(alpha), _ptr(accept_prob), _ptr(status), B, K, float(lam), _ptr(out),
+                                       _stream(stream)), "ssd_alpha_update")
+    return out
+
+
+def ssd_fallback_bstar(h: float, alpha: float, K: int, L_target: float, L_primary: float, L_fast: float,
+                       E_fast: float, b_max: int):
+    """(b*, choice[b_max] as a numpy uint8 array) of the batch-size fallback policy (host)."""
+    import numpy as np
+    choice = np.zeros(b_max, np.uint8)
+    r = load().ssd_fallback_bstar(float(h), float(alpha), int(K), float(L_target), float(L_primary),
+                                  float(L_fast), float(E_fast), int(b_max), C.c_void_p(choice.ctypes.data))
+    if r < 0:
+        raise SsdError("ssd_fallback_bstar: arguments out of range")
+    return int(r), choice
+
+
+def ssd_prespeculate(key_logits: torch.Tensor, T: float, F_next: torch.Tensor, C_coef: float, next_budget: int,
+                     uniforms: torch.Tensor, workspace: Optional["Workspace"] = None, payload=None, stream=None):
+    """Draw the K-token payload of every cache key (see ssd.h); returns (payload, status)."""
+    B, n_keys, K, V = key_logits.shape
+    dev = key_logits.device
+    dt = _logit_dtype(key_logits)
+    _need(key_logits, "key_logits", key_logits.dtype, (B, n_keys, K, V), dev)
+    _need(F_next, "F_next", torch.int32, (B * n_keys, K + 1), dev)
+    _need(uniforms, "uniforms", torch.float32, (B, n_keys, K), dev)
+    if payload is None:
+        payload = torch.empty((B, n_keys, K), dtype=torch.int32, device=dev)
+    _need(payload, "payload", torch.int32, (B, n_keys, K), dev)
+    status = torch.empty(B * n_keys, dtype=torch.int32, device=dev)
+    if workspace is None:
+        workspace = default_workspace(dev, B * n_keys, K, V, dt)
+    with torch.cuda.device(dev):
+        _check(load().ssd_prespeculate(_ptr(key_logits), dt, B, n_keys, K, V, float(T), _ptr(F_next),
+                                       float(C_coef), int(next_budget), _ptr(uniforms), _ptr(payload),
+                                       _ptr(status), workspace.ptr(), workspace.nbytes, _stream(stream)),
+               "ssd_prespeculate")
+    return payload, status
 
 
 @dataclass

@@ -28,6 +28,39 @@ __global__ void fanout_kernel(const float* __restrict__ alpha, int B, int K, int
              F + static_cast<long long>(b) * (K + 1));
 }
 
+__global__ void fanout_power_kernel(const float* __restrict__ alpha, int B, int K, int budget, int q,
+                                    int32_t* __restrict__ F) {
+  const int b = blockIdx.x * blockDim.x + threadIdx.x;
+  if (b >= B) return;
+  fanout_row_power(alpha[b], K, budget, q, F + static_cast<long long>(b) * (K + 1));
+}
+
+// ---------------------------------------------------------------------------
+// Per-row acceptance from history: alpha' = (1 - lambda) alpha + lambda *
+// mean_j a_j, in double with every operation rounded on its own, then
+// rounded to float.  Invalid rows and rows with a NaN a_j keep their alpha.
+// ---------------------------------------------------------------------------
+__global__ void alpha_update_kernel(const float* __restrict__ alpha, const float* __restrict__ accept_prob,
+                                    const int32_t* __restrict__ status, int B, int K, double lambda,
+                                    float* __restrict__ alpha_out) {
+  const int b = blockIdx.x * blockDim.x + threadIdx.x;
+  if (b >= B) return;
+  bool ok = (status[b] & SSD_ROW_INVALID) == 0;
+  double s = 0.0;
+  for (int j = 0; j < K; ++j) {
+    const double a = static_cast<double>(accept_prob[static_cast<long long>(b) * K + j]);
+    if (a != a) ok = false;
+    s = __dadd_rn(s, a);
+  }
+  if (!ok) {
+    alpha_out[b] = alpha[b];
+    return;
+  }
+  const double mean = __ddiv_rn(s, static_cast<double>(K));
+  const double keep = __dmul_rn(__dsub_rn(1.0, lambda), static_cast<double>(alpha[b]));
+  alpha_out[b] = __double2float_rn(__dadd_rn(keep, __dmul_rn(lambda, mean)));
+}
+
 // ---------------------------------------------------------------------------
 // Cache build: offsets = prefix sums of F; tokens copied per segment.
 // ---------------------------------------------------------------------------
@@ -405,19 +438,16 @@ ssd_status ssd_verify(const void* target_logits, const void* draft_logits, const
   return launch(a, dtype, V % VE == 0, units, B, static_cast<cudaStream_t>(stream));
 }
 
-ssd_status ssd_saguaro_reweight(const void* draft_logits, int dtype, int B, int K, int V, float T, const int32_t* F,
+}  // extern "C"
+
+namespace ssd {
+// The draft-side pass behind ssd_saguaro_reweight and ssd_prespeculate; the
+// per-position outputs topf_tokens, offsets, Z and q_lse may be null here.
+static ssd_status reweight_impl(const void* draft_logits, int dtype, int B, int K, int V, float T, const int32_t* F,
                                 float C, int budget, const void* guess_logits, int64_t guess_row_stride,
                                 const float* u_draft, int32_t* topf_tokens, int32_t* offsets, float* Z,
                                 float* q_lse, int32_t* draft_tokens_out, int32_t* status, void* workspace,
                                 size_t ws_bytes, void* stream) {
-  if (dtype != SSD_DTYPE_BF16 && dtype != SSD_DTYPE_FP32) return SSD_ERR_DTYPE;
-  if (B < 0 || K < 1 || K > SSD_MAX_K || V < 1) return SSD_ERR_INVALID_ARG;
-  if (!(T >= 0.f) || isinf(T) || !(C > 0.f && C <= 1.f)) return SSD_ERR_INVALID_ARG;
-  if (budget < 0 || budget > SSD_MAX_BUDGET || budget > V) return SSD_ERR_INVALID_ARG;
-  if (draft_tokens_out && !u_draft) return SSD_ERR_INVALID_ARG;
-  if (guess_logits && guess_row_stride < V) return SSD_ERR_INVALID_ARG;
-  if (B == 0) return SSD_OK;
-  if (!draft_logits || !F || !topf_tokens || !offsets || !Z || !q_lse || !status) return SSD_ERR_INVALID_ARG;
   if (!aligned16(draft_logits) || (guess_logits && !aligned16(guess_logits))) return SSD_ERR_ALIGNMENT;
   const WsLayout wl = ws_layout(B, K, V, dtype);
   if (!workspace || ws_bytes < wl.total) return SSD_ERR_WORKSPACE;
@@ -453,6 +483,91 @@ ssd_status ssd_saguaro_reweight(const void* draft_logits, int dtype, int B, int 
   a.draws = draws ? 1 : 0;
   const long long draw_units = draws ? static_cast<long long>(B) * K : 0;
   return launch(a, dtype, aligned, units, draw_units, static_cast<cudaStream_t>(stream));
+}
+}  // namespace ssd
+
+extern "C" {
+
+ssd_status ssd_saguaro_reweight(const void* draft_logits, int dtype, int B, int K, int V, float T, const int32_t* F,
+                                float C, int budget, const void* guess_logits, int64_t guess_row_stride,
+                                const float* u_draft, int32_t* topf_tokens, int32_t* offsets, float* Z,
+                                float* q_lse, int32_t* draft_tokens_out, int32_t* status, void* workspace,
+                                size_t ws_bytes, void* stream) {
+  if (dtype != SSD_DTYPE_BF16 && dtype != SSD_DTYPE_FP32) return SSD_ERR_DTYPE;
+  if (B < 0 || K < 1 || K > SSD_MAX_K || V < 1) return SSD_ERR_INVALID_ARG;
+  if (!(T >= 0.f) || isinf(T) || !(C > 0.f && C <= 1.f)) return SSD_ERR_INVALID_ARG;
+  if (budget < 0 || budget > SSD_MAX_BUDGET || budget > V) return SSD_ERR_INVALID_ARG;
+  if (draft_tokens_out && !u_draft) return SSD_ERR_INVALID_ARG;
+  if (guess_logits && guess_row_stride < V) return SSD_ERR_INVALID_ARG;
+  if (B == 0) return SSD_OK;
+  if (!draft_logits || !F || !topf_tokens || !offsets || !Z || !q_lse || !status) return SSD_ERR_INVALID_ARG;
+  return reweight_impl(draft_logits, dtype, B, K, V, T, F, C, budget, guess_logits, guess_row_stride, u_draft,
+                       topf_tokens, offsets, Z, q_lse, draft_tokens_out, status, workspace, ws_bytes, stream);
+}
+
+ssd_status ssd_prespeculate(const void* key_logits, int dtype, int B, int n_keys, int K, int V, float T,
+                            const int32_t* F_next, float C, int next_budget, const float* uniforms,
+                            int32_t* payload, int32_t* status, void* workspace, size_t ws_bytes, void* stream) {
+  if (dtype != SSD_DTYPE_BF16 && dtype != SSD_DTYPE_FP32) return SSD_ERR_DTYPE;
+  if (B < 0 || n_keys < 0 || K < 1 || K > SSD_MAX_K || V < 1) return SSD_ERR_INVALID_ARG;
+  if (!(T >= 0.f) || isinf(T) || !(C > 0.f && C <= 1.f)) return SSD_ERR_INVALID_ARG;
+  if (next_budget < 0 || next_budget > SSD_MAX_BUDGET || next_budget > V) return SSD_ERR_INVALID_ARG;
+  const long long rows = static_cast<long long>(B) * n_keys;
+  if (rows > 0x7FFFFFFFLL) return SSD_ERR_INVALID_ARG;
+  if (rows == 0) return SSD_OK;
+  if (!key_logits || !F_next || !uniforms || !payload || !status) return SSD_ERR_INVALID_ARG;
+  return reweight_impl(key_logits, dtype, static_cast<int>(rows), K, V, T, F_next, C, next_budget, nullptr, 0,
+                       uniforms, nullptr, nullptr, nullptr, nullptr, payload, status, workspace, ws_bytes, stream);
+}
+
+ssd_status ssd_fanout_plan_power(const float* alpha, int B, int K, int budget, int gamma_eighths, int32_t* F,
+                                 void* stream) {
+  if (B < 0 || K < 1 || K > SSD_MAX_K || budget < 0 || budget > SSD_MAX_BUDGET) return SSD_ERR_INVALID_ARG;
+  if (gamma_eighths < 1 || gamma_eighths > 8) return SSD_ERR_INVALID_ARG;
+  if (B == 0) return SSD_OK;
+  if (!F || !alpha) return SSD_ERR_INVALID_ARG;
+  fanout_power_kernel<<<(B + 127) / 128, 128, 0, static_cast<cudaStream_t>(stream)>>>(alpha, B, K, budget,
+                                                                                     gamma_eighths, F);
+  return cudaGetLastError() == cudaSuccess ? SSD_OK : SSD_ERR_CUDA;
+}
+
+ssd_status ssd_alpha_update(const float* alpha, const float* accept_prob, const int32_t* status, int B, int K,
+                            double lambda, float* alpha_out, void* stream) {
+  if (B < 0 || K < 1 || K > SSD_MAX_K || !(lambda >= 0.0 && lambda <= 1.0)) return SSD_ERR_INVALID_ARG;
+  if (B == 0) return SSD_OK;
+  if (!alpha || !accept_prob || !status || !alpha_out) return SSD_ERR_INVALID_ARG;
+  alpha_update_kernel<<<(B + 127) / 128, 128, 0, static_cast<cudaStream_t>(stream)>>>(alpha, accept_prob, status, B,
+                                                                                     K, lambda, alpha_out);
+  return cudaGetLastError() == cudaSuccess ? SSD_OK : SSD_ERR_CUDA;
+}
+
+// Batch-size fallback policy ([ZH] section 2 challenge 3; [NL] section 3C).
+// Host arithmetic in double: per-row tokens of a round E_p = sum_{i<=K}
+// alpha^i with the primary speculator (a hit, or a miss it serves), E_fast
+// for a miss served by the fast one; a round lasts L_target plus the
+// fallback's latency with probability 1 - h^b (some row of the batch missed).
+int ssd_fallback_bstar(double h, double alpha, int K, double L_target, double L_primary, double L_fast,
+                       double E_fast, int b_max, uint8_t* choice) {
+  if (!(h >= 0.0 && h <= 1.0) || !(alpha >= 0.0 && alpha <= 1.0) || K < 0 || b_max < 1 || !(L_target > 0.0) ||
+      !(L_primary >= 0.0) || !(L_fast >= 0.0) || !(E_fast >= 0.0))
+    return -1;
+  double E_p = 0.0, power = 1.0;
+  for (int i = 0; i <= K; ++i) {
+    E_p += power;
+    power *= alpha;
+  }
+  int first = b_max + 1;
+  double all_hit = 1.0;
+  for (int b = 1; b <= b_max; ++b) {
+    all_hit *= h;
+    const double wait = 1.0 - all_hit;
+    const double primary = E_p / (L_target + wait * L_primary);
+    const double fast = (h * E_p + (1.0 - h) * E_fast) / (L_target + wait * L_fast);
+    const bool use_fast = fast > primary;
+    if (choice) choice[b - 1] = use_fast ? 1 : 0;
+    if (use_fast && first > b_max) first = b;
+  }
+  return first;
 }
 
 }  // extern "C"

@@ -431,6 +431,67 @@ __device__ __forceinline__ void fanout_row(float alpha_f, int K, int budget, int
 }
 
 
+// Power-law plan ([ZH] section 2 challenge 1, the acceptance's power law;
+// [NL] section 3A, a geometric series): F_k proportional to P(k)^gamma,
+// gamma = q / 8, the optimum when an outcome's hit rate given F guesses
+// follows a power-law curve.  alpha^gamma and (1 - alpha)^gamma are the
+// eighth root (three correctly rounded square roots) raised to the q-th power
+// by q - 1 rounded products; weights w_k = a^k c (k < K), w_K = a^K; quotas
+// budget * w_k / W with W summed in k order; largest remainder as in
+// fanout_row.  Every operation is rounded on its own, so the plan is the same
+// integers on every device and host.  q = 8 is fanout_row's geometric plan.
+__device__ __forceinline__ double eighth_power(double x, int q) {
+  const double r = __dsqrt_rn(__dsqrt_rn(__dsqrt_rn(x)));
+  double y = r;
+  for (int i = 1; i < q; ++i) y = __dmul_rn(y, r);
+  return y;
+}
+
+__device__ __forceinline__ void fanout_row_power(float alpha_f, int K, int budget, int q, int32_t* f) {
+  if (q == 8) {
+    fanout_row(alpha_f, K, budget, SSD_FANOUT_GEOMETRIC, f);
+    return;
+  }
+  const double al = static_cast<double>(alpha_f);
+  if (!(al >= 0.0 && al <= 1.0)) {
+    f[0] = -1;
+    for (int k = 1; k <= K; ++k) f[k] = 0;
+    return;
+  }
+  const double a = eighth_power(al, q), c = eighth_power(__dsub_rn(1.0, al), q);
+  double w[SSD_MAX_K + 1], frac[SSD_MAX_K + 1];
+  bool taken[SSD_MAX_K + 1];
+  double run = 1.0, W = 0.0;
+  for (int k = 0; k < K; ++k) {
+    w[k] = __dmul_rn(run, c);
+    run = __dmul_rn(run, a);
+  }
+  w[K] = run;
+  for (int k = 0; k <= K; ++k) W = __dadd_rn(W, w[k]);
+  long long assigned = 0;
+  for (int k = 0; k <= K; ++k) {
+    const double quota = __ddiv_rn(__dmul_rn(static_cast<double>(budget), w[k]), W);
+    const double fl = floor(quota);
+    f[k] = static_cast<int32_t>(fl);
+    frac[k] = __dsub_rn(quota, fl);
+    taken[k] = false;
+    assigned += f[k];
+  }
+  long long rem = budget - assigned;
+  while (rem > 0) {
+    int best = -1;
+    for (int k = 0; k <= K; ++k)
+      if (!taken[k] && (best < 0 || frac[k] > frac[best])) best = k;
+    if (best < 0) {
+      for (int k = 0; k <= K; ++k) taken[k] = false;
+      continue;
+    }
+    taken[best] = true;
+    f[best] += 1;
+    --rem;
+  }
+}
+
 // Ring of bulk copies that streams one slice of up to two rows of a unit
 // through shared memory, chunk by chunk (CV 16-byte vectors per row per
 // chunk, ST stages).  Thread 0 issues and polls; the other threads sleep in the
@@ -1101,7 +1162,7 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) ssd_stats_kernel(const _
   int32_t* segdst = nullptr;
   if (verify) {
     if (a.c_tokens && !plan_bad) segdst = a.c_tokens + static_cast<long long>(b) * a.budget + seg_off;
-  } else if (!plan_bad) {
+  } else if (!plan_bad && a.topf_tokens) {
     segdst = a.topf_tokens + static_cast<long long>(b) * a.budget + seg_off;
   }
   if (segdst && has_plan)
@@ -1111,8 +1172,8 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) ssd_stats_kernel(const _
     if (!verify && j < K) {
       const long long o = static_cast<long long>(b) * K + j;
       const float qlse = kGreedy ? MQ : (MQ * cT + log2f(SQ)) * 0.6931471805599453f;
-      a.Z[o] = valid ? Z : __int_as_float(0x7FC00000);
-      a.q_lse[o] = valid ? qlse : __int_as_float(0x7FC00000);
+      if (a.Z) a.Z[o] = valid ? Z : __int_as_float(0x7FC00000);
+      if (a.q_lse) a.q_lse[o] = valid ? qlse : __int_as_float(0x7FC00000);
       if (a.draft_tokens && (!valid || !a.draws)) a.draft_tokens[o] = valid ? sm.argQ : -1;
     }
     UnitState st;
@@ -1189,10 +1250,12 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) ssd_stats_kernel(const _
     } else if (lane == 0) {
       const bool pbad = (fl & SSD_ROW_BAD_PLAN) != 0;
       int off = 0;
-      a.offsets[static_cast<long long>(b) * (K + 2)] = 0;
-      for (int k = 0; k <= K; ++k) {
-        off += pbad ? 0 : sm.s_F[k];
-        a.offsets[static_cast<long long>(b) * (K + 2) + k + 1] = off;
+      if (a.offsets) {
+        a.offsets[static_cast<long long>(b) * (K + 2)] = 0;
+        for (int k = 0; k <= K; ++k) {
+          off += pbad ? 0 : sm.s_F[k];
+          a.offsets[static_cast<long long>(b) * (K + 2) + k + 1] = off;
+        }
       }
       if (!a.draws) a.status[b] = fl;
       else {

@@ -676,3 +676,137 @@ def test_log_normalisers_match_library_logsumexp():
     out = oracle.verify(lp, lq, np.zeros((2, K), np.int32), np.zeros((2, K + 1), np.float32), T, n_threads=1)
     np.testing.assert_allclose(out["p_lse"], logsumexp(lp.astype(np.float64) / T, axis=2), rtol=1e-14, atol=0)
     np.testing.assert_allclose(out["q_lse"], logsumexp(lq.astype(np.float64) / T, axis=2), rtol=1e-14, atol=0)
+
+
+# ---------------------------------------------------------------------------
+# Fan-out variants: the power-law plan (gamma = q/8) and the per-row alpha
+# update from history.
+# ---------------------------------------------------------------------------
+def power_quotas(alpha, K, budget, gamma):
+    P = np.array([alpha ** k * (1 - alpha) for k in range(K)] + [alpha ** K])
+    w = P ** gamma
+    return budget * w / w.sum()
+
+
+def test_power_plan_gamma_one_is_the_geometric_plan():
+    rng = np.random.default_rng(2)
+    for _ in range(200):
+        K, budget, alpha = int(rng.integers(1, 12)), int(rng.integers(0, 300)), float(np.float32(rng.random()))
+        np.testing.assert_array_equal(oracle.fanout_plan_power(alpha, K, budget, 8), oracle.fanout_plan(alpha, K, budget))
+
+
+def test_power_plan_sum_rank_quota_bounds_and_ratio():
+    """Sum = budget; every F_k is the floor or the ceiling of its quota
+    budget * P(k)^gamma / sum P^gamma (quotas computed here with pow); F is
+    non-increasing in quota rank; successive real quotas have ratio alpha^gamma."""
+    rng = np.random.default_rng(3)
+    for _ in range(400):
+        K = int(rng.integers(1, 12))
+        budget = int(rng.integers(0, 300))
+        alpha = float(np.float32(rng.uniform(0.01, 0.99)))
+        q = int(rng.integers(1, 8))
+        F = oracle.fanout_plan_power(alpha, K, budget, q)
+        Q = power_quotas(alpha, K, budget, q / 8)
+        assert F.sum() == budget and np.all(F >= 0)
+        assert np.all(np.abs(F - Q) < 1.0 + 1e-9), (alpha, K, budget, q, F, Q)
+        for a, b in itertools.combinations(range(K + 1), 2):
+            if Q[a] > Q[b] + 1e-9:
+                assert F[a] >= F[b]
+        for k in range(K - 1):
+            if budget > 0:
+                assert abs(Q[k + 1] / Q[k] - alpha ** (q / 8)) < 1e-12
+
+
+def test_power_plan_flattens_as_gamma_falls():
+    """A smaller gamma moves branches from the most likely outcome to the
+    least likely one: as gamma grows, the most likely outcome never loses a
+    branch and the least likely never gains one."""
+    for alpha in (0.3, 0.6, 0.85):
+        P = [alpha ** k * (1 - alpha) for k in range(6)] + [alpha ** 6]
+        hi, lo = int(np.argmax(P)), int(np.argmin(P))
+        plans = [oracle.fanout_plan_power(alpha, 6, 96, q) for q in range(1, 9)]
+        for a, b in zip(plans, plans[1:]):
+            assert b[hi] >= a[hi] and b[lo] <= a[lo]
+
+
+def test_power_plan_is_the_hit_optimal_split_under_a_power_law_hit_curve():
+    """The reading behind gamma: with a hit curve h(F) = 1 - (1 + F)^-beta per
+    outcome, maximising sum_k P(k) h(F_k) under sum F = budget (solved
+    numerically here, over real F) gives F ~ P^(1/(1+beta)) up to the +1
+    offset; for a large budget the integer plan at gamma = 1/(1+beta) must be
+    within a few branches of that optimum."""
+    from scipy.optimize import minimize
+    for alpha, beta, q in ((0.7, 1.0, 4), (0.6, 1.0 / 3.0, 6), (0.8, 3.0, 2)):
+        K, budget = 6, 4096
+        P = np.array([alpha ** k * (1 - alpha) for k in range(K)] + [alpha ** K])
+
+        def neg(x):
+            F = budget * np.exp(x) / np.exp(x).sum()
+            return -np.sum(P * (1 - (1 + F) ** -beta))
+
+        res = minimize(neg, np.log(P ** (q / 8)), method="Nelder-Mead",
+                       options=dict(xatol=1e-10, fatol=1e-14, maxiter=20000))
+        Fopt = budget * np.exp(res.x) / np.exp(res.x).sum()
+        F = oracle.fanout_plan_power(alpha, K, budget, q)
+        assert abs(q / 8 - 1 / (1 + beta)) < 1e-12
+        assert np.max(np.abs(F - Fopt)) < 0.01 * budget, (F, Fopt)
+
+
+def test_alpha_update_closed_forms():
+    rng = np.random.default_rng(4)
+    B, K = 16, 5
+    alpha = rng.random(B).astype(np.float32)
+    ap = rng.random((B, K)).astype(np.float32)
+    st = np.zeros(B, np.int32)
+    st[3] = oracle.ROW_BAD_TOKEN
+    ap[5, 2] = np.nan
+    st[6] = oracle.ROW_NEAR_TIE          # informational: still updated
+    full = oracle.alpha_update(alpha, ap, st, 1.0)
+    none = oracle.alpha_update(alpha, ap, st, 0.0)
+    half = oracle.alpha_update(alpha, ap, st, 0.5)
+    keep = np.zeros(B, bool)
+    keep[[3, 5]] = True
+    np.testing.assert_array_equal(full[keep], alpha[keep])
+    np.testing.assert_array_equal(none, alpha)
+    mean = ap.astype(np.float64).mean(axis=1)
+    np.testing.assert_allclose(full[~keep], mean[~keep].astype(np.float32), rtol=0, atol=6e-8)
+    np.testing.assert_allclose(half[~keep], (0.5 * alpha + 0.5 * mean)[~keep], rtol=0, atol=6e-8)
+
+
+# ---------------------------------------------------------------------------
+# The batch-size fallback policy b*: the crossing in closed form.
+# ---------------------------------------------------------------------------
+def bstar_closed_form(h, alpha, K, Lt, Lp, Lf, Ef, b_max):
+    """The fast fallback wins iff m = 1 - h^b exceeds
+    m* = (1-h) Lt (Ep - Ef) / (Lp (h Ep + (1-h) Ef) - Ep Lf)  (denominator > 0)."""
+    Ep = sum(alpha ** i for i in range(K + 1))
+    den = Lp * (h * Ep + (1 - h) * Ef) - Ep * Lf
+    if den <= 0:
+        return b_max + 1
+    mstar = (1 - h) * Lt * (Ep - Ef) / den
+    for b in range(1, b_max + 1):
+        if 1 - h ** b > mstar * (1 + 1e-12) + 1e-15:
+            return b
+    return b_max + 1
+
+
+def test_fallback_bstar_matches_the_closed_form():
+    rng = np.random.default_rng(5)
+    for _ in range(300):
+        h = float(rng.uniform(0.5, 0.999))
+        alpha = float(rng.uniform(0.3, 0.9))
+        K = int(rng.integers(2, 9))
+        Lt, Lp = float(rng.uniform(5, 30)), float(rng.uniform(0.5, 20))
+        Lf, Ef = float(rng.uniform(0.0, 0.2)), 1.0
+        bs, choice = oracle.fallback_bstar(h, alpha, K, Lt, Lp, Lf, Ef, 512)
+        assert bs == bstar_closed_form(h, alpha, K, Lt, Lp, Lf, Ef, 512)
+        # below b* the primary speculator, from b* on the fast one
+        assert np.all(choice[:bs - 1] == 0) and np.all(choice[bs - 1:] == 1)
+
+
+def test_fallback_small_batches_primary_large_batches_fast():
+    """The pages' qualitative rule: a batch of one keeps the primary
+    speculator when its fallback is cheap relative to a round; very large
+    batches switch to the fast one."""
+    bs, choice = oracle.fallback_bstar(0.95, 0.7, 6, 20.0, 2.0, 0.05, 1.0, 4096)
+    assert choice[0] == 0 and 1 < bs <= 4096 and choice[-1] == 1
