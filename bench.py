@@ -2,24 +2,27 @@
 """Benchmark of the fused verify + speculation-cache step (libssd) on B200.
 
 One step = the whole hot path over one batch: the fan-out plan and the fused
-verify kernel (softmax statistics, top-F, Saguaro reweighting, accept test,
-residual bonus draw, cache build and lookup).  Inputs are seeded synthetic
-Zipf logits, generated on the host, resident in HBM before timing starts; two
-input copies rotate, each larger than the 126 MB L2.
+verify (softmax statistics, top-F, Saguaro reweighting, accept test, residual
+bonus draw, cache build and lookup).  Inputs are seeded synthetic Zipf
+logits, generated on the host and resident in HBM before timing starts;
+enough input copies rotate that their total exceeds twice the 126 MB L2.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+    python bench.py --workload zipf_b256_k8_v151936_bf16_sweep --sweep
+        # one line per (T, fan-out mode, C): rows/s, GB/s, hit rate
+    python bench.py --workload zipf_b512_k4_v128256_bf16_miss --unfused
+        # the five-call step (plan, reweight, verify, cache build, lookup)
     python bench.py --impl reference ...   # the fp64 CPU oracle on host cores
 
 Under torchrun (N > 1) every rank runs the same per-GPU workload on its own
 rows (weak scaling, no collective on the data path); the step time is the
-maximum over ranks.  Rank 0 prints one JSON line.
+maximum over ranks.  Rank 0 prints one JSON line (per sweep point).
 """
 import argparse
 import hashlib
 import json
 import os
 import statistics
-import subprocess
 import sys
 import threading
 import time
@@ -34,11 +37,14 @@ L2_BYTES = 126 * 1024 * 1024
 KERNEL_SOURCES = ["speculative_decoding_verify_ssd_b200/csrc/ssd_kernels.cuh",
                   "speculative_decoding_verify_ssd_b200/csrc/ssd_device.cuh",
                   "speculative_decoding_verify_ssd_b200/csrc/ssd_api.cu"]
-
+GRAPH_CALLS = 200  # verify calls captured per CUDA graph; the timed region replays graphs summing to --steps
 
 # ssd_verify launches ssd_stats_kernel (softmax statistics, top-F, accept test,
 # row decision) and then ssd_draw_kernel (residual / bonus draw, cache lookup).
 KERNELS_PER_VERIFY = 2
+# the unfused step: fan-out plan, reweight (its statistics kernel; no draft
+# draw), verify without a cache (2), cache build, cache lookup
+KERNELS_PER_UNFUSED = 6
 
 
 def ssd_step_kernels():
@@ -69,7 +75,7 @@ def measured_peaks():
 
 
 def recorded_traffic(workload):
-    """DRAM bytes per launch of the verify kernel from a committed ncu
+    """DRAM bytes per launch of the verify kernels from a committed ncu
     summary, only if it was taken on the current kernel sources."""
     try:
         with open(os.path.join(ROOT, "profiles", "verify_traffic.json")) as f:
@@ -83,57 +89,53 @@ def recorded_traffic(workload):
 
 
 class ClockSampler:
-    """nvidia-smi clock / throttle sampling during the timed region."""
+    """SM clock, max clock and throttle reasons sampled through NVML every
+    few milliseconds while the timed region runs."""
 
-    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = (("hw_slowdown", 0x8), ("hw_thermal_slowdown", 0x40), ("sw_thermal_slowdown", 0x20),
+               ("sw_power_cap", 0x4))
 
     def __init__(self, index):
         self.index = index
-        self.proc = None
-        self.lines = []
+        self.samples = []
+        self.reasons = set()
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._thr = None
 
     def start(self):
         try:
-            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.Q}",
-                                          "--format=csv,noheader,nounits", "-lms", "100"],
-                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-            self.thr = threading.Thread(target=self._read, daemon=True)
-            self.thr.start()
+            import pynvml
+            pynvml.nvmlInit()
+            h = pynvml.nvmlDeviceGetHandleByIndex(self.index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
         except Exception:
-            self.proc = None
+            return
 
-    def _read(self):
-        for line in self.proc.stdout:
-            self.lines.append(line.strip())
+        def loop():
+            while not self._stop.is_set():
+                try:
+                    self.samples.append(pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM))
+                    r = pynvml.nvmlDeviceGetCurrentClocksThrottleReasons(h)
+                    for name, bit in self.REASONS:
+                        if r & bit:
+                            self.reasons.add(name)
+                except Exception:
+                    pass
+                time.sleep(0.002)
+
+        self._thr = threading.Thread(target=loop, daemon=True)
+        self._thr.start()
 
     def stop(self):
-        if self.proc is None:
+        if self._thr is None:
             return None
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except Exception:
-            self.proc.kill()
-        sm, mx, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
-            parts = [p.strip() for p in ln.split(",")]
-            if len(parts) < 9:
-                continue
-            try:
-                sm.append(float(parts[1]))
-                mx = float(parts[2])
-            except ValueError:
-                continue
-            for name, val in zip(names, parts[5:9]):
-                if val.lower().startswith("active"):
-                    reasons.add(name)
-        if not sm:
+        self._stop.set()
+        self._thr.join(timeout=2)
+        if not self.samples:
             return None
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
-                "samples": len(sm)}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples), "source": "nvml, every 2 ms"}
 
 
 def rank_workload(w, rank):
@@ -171,6 +173,96 @@ def algorithmic_bytes(w):
     return logits, logits + inputs + outputs
 
 
+def n_rotating_copies(logit_bytes):
+    """Input copies so that the rotation exceeds twice the L2 (small
+    workloads would otherwise be served from L2), within 4 GB."""
+    n = max(2, -(-2 * L2_BYTES // logit_bytes))
+    return int(min(n, max(2, (4 << 30) // logit_bytes)))
+
+
+def make_sets(w, n_copies, dev, ssd, synth):
+    import torch
+
+    def dev_logits(x):
+        if x.dtype == np.uint16:
+            return torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).to(dev)
+        return torch.from_numpy(x).to(dev)
+
+    sets, host_first = [], None
+    for c in range(n_copies):
+        g = synth.generate(w.replace(seed=w.seed + 104729 * c))
+        if c == 0:
+            host_first = g
+        sets.append(dict(t=dev_logits(g["target"]), d=dev_logits(g["draft"]),
+                         u=torch.from_numpy(g["uniforms"]).to(dev), u_draft=torch.from_numpy(g["u_draft"]).to(dev)))
+        del g
+    return sets, host_first
+
+
+def draw_tokens(w, sets, dev, ssd):
+    """Draft tokens from the draft side's own Saguaro sampler (d_j ~ q'_j)."""
+    import torch
+    for s in sets:
+        s["alpha"] = torch.full((w.B,), w.alpha, dtype=torch.float32, device=dev)
+        s["F"] = ssd.ssd_fanout_plan(s["alpha"], w.K, w.budget, w.fanout_mode)
+        rw = ssd.ssd_saguaro_reweight(s["d"], w.T, s["F"], w.C, w.budget, u_draft=s["u_draft"])
+        s["tok"] = rw.draft_tokens
+    torch.cuda.synchronize()
+
+
+def time_steps(step, steps, warmup, dev, world, dist, sampler_index):
+    """Warm up, capture CUDA graphs of up to GRAPH_CALLS steps, and time
+    exactly `steps` steps (graph replays summing to `steps`) with CUDA events
+    on the launching stream.  Returns (total_ms, per-step ms of each replay,
+    clocks)."""
+    import torch
+    for i in range(warmup):
+        step(i)
+    torch.cuda.synchronize()
+    per_graph = min(steps, GRAPH_CALLS)
+    full, rest = divmod(steps, per_graph)
+    graphs = []
+    cap = torch.cuda.Stream(dev)
+    cap.wait_stream(torch.cuda.current_stream(dev))
+    for n in ([per_graph] if full else []) + ([rest] if rest else []):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(cap):
+            with torch.cuda.graph(g, stream=cap, capture_error_mode="thread_local"):
+                for i in range(n):
+                    step(i)
+        graphs.append((g, n))
+    torch.cuda.synchronize()
+    for g, _ in graphs:
+        g.replay()
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream(dev)
+    plan = [graphs[0]] * full + ([graphs[-1]] if rest else [])
+    sampler = ClockSampler(sampler_index) if sampler_index is not None else None
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    if sampler:
+        sampler.start()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    marks = []
+    start.record(stream)
+    for g, n in plan:
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        g.replay()
+        e1.record(stream)
+        marks.append((e0, e1, n))
+    end.record(stream)
+    torch.cuda.synchronize()
+    clocks = sampler.stop() if sampler else None
+    if world > 1:
+        dist.barrier()
+    total_ms = start.elapsed_time(end)
+    per_step = [a.elapsed_time(b) / n for a, b, n in marks]
+    del graphs, plan
+    return total_ms, per_step, clocks
+
+
 def run_ssd(args, rank, world, local_rank):
     import torch
     from speculative_decoding_verify_ssd_b200 import binding as ssd
@@ -179,135 +271,95 @@ def run_ssd(args, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
     ssd.load()
-    w = synth.WORKLOADS[args.workload]
-    w_rank = rank_workload(w, rank)
-    logit_bytes, alg_bytes = algorithmic_bytes(w)
-    n_copies = max(2, -(-2 * L2_BYTES // logit_bytes))
-    n_copies = min(n_copies, 8)
-
-    def dev_logits(x):
-        if x.dtype == np.uint16:
-            return torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).to(dev)
-        return torch.from_numpy(x).to(dev)
-
-    sets = []
-    host_first = None
-    for c in range(n_copies):
-        g = synth.generate(w_rank.replace(seed=w_rank.seed + 104729 * c))
-        if c == 0:
-            host_first = g
-        t, d = dev_logits(g["target"]), dev_logits(g["draft"])
-        alpha = torch.from_numpy(g["alpha"]).to(dev)
-        u = torch.from_numpy(g["uniforms"]).to(dev)
-        F = ssd.ssd_fanout_plan(alpha, w.K, w.budget, w.fanout_mode)
-        # Draft tokens come from the draft side's own Saguaro sampler.
-        rw = ssd.ssd_saguaro_reweight(d, w.T, F, w.C, w.budget,
-                                      u_draft=torch.from_numpy(g["u_draft"]).to(dev))
-        sets.append(dict(t=t, d=d, alpha=alpha, u=u, tok=rw.draft_tokens))
-        del g
-    torch.cuda.synchronize()
-    ws = ssd.Workspace(w.B, w.K, dev, w.V, ssd.DTYPE_BF16 if w.dtype == "bf16" else ssd.DTYPE_FP32)
-    outs = [ssd.alloc_verify_result(w.B, w.K, w.budget, dev, True) for _ in range(n_copies)]
-
-    def step(i):
-        # One launch: the fan-out plan is computed inside the fused kernel from alpha.
-        s = sets[i % n_copies]
-        ssd.ssd_verify(s["t"], s["d"], s["tok"], s["u"], w.T, alpha=s["alpha"], fanout_mode=w.fanout_mode,
-                       C_coef=w.C, budget=w.budget, cache=True, fallback_seed=w_rank.fallback_seed,
-                       workspace=ws, out=outs[i % n_copies])
-
-    for i in range(args.warmup):
-        step(i)
-    torch.cuda.synchronize()
-    # The timed loop is one CUDA graph of `steps` back-to-back launches, so
-    # host launch overhead never starves the GPU.
-    graph = torch.cuda.CUDAGraph()
-    cap = torch.cuda.Stream(dev)
-    cap.wait_stream(torch.cuda.current_stream(dev))
-    with torch.cuda.stream(cap):
-        with torch.cuda.graph(graph, stream=cap, capture_error_mode="thread_local"):
-            for i in range(args.steps):
-                step(i)
-    torch.cuda.synchronize()
-    for _ in range(2):
-        graph.replay()
-    torch.cuda.synchronize()
-    stream = torch.cuda.current_stream(dev)
-
     dist = None
     if world > 1:
         import torch.distributed as dist
-        dist.barrier()
-    sampler = ClockSampler(local_rank) if rank == 0 else None
-    if sampler:
-        sampler.start()
-        time.sleep(0.3)
-    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    reps = max(1, args.repeat)
-    per_rep = []
-    torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
-    start.record(stream)
-    for r in range(reps):
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        graph.replay()
-        e1.record(stream)
-        per_rep.append((e0, e1))
-    end.record(stream)
-    torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
-    clocks = sampler.stop() if sampler else None
-    total_ms = start.elapsed_time(end)
-    steps_done = args.steps * reps
-    # the graph holds `steps` verify calls back to back: per-step time = replay time / steps
-    kernel_ms = [a.elapsed_time(b) / args.steps for a, b in per_rep]
-    if world > 1:
-        total_ms = max_over_ranks(total_ms, dist, dev)
-    ms_per_step = total_ms / steps_done
-    rows_per_s = job_rows_per_s(world, w.B, steps_done, total_ms)
-    del graph
+    w0 = synth.WORKLOADS[args.workload]
+    w_rank = rank_workload(w0, rank)
+    logit_bytes, alg_bytes = algorithmic_bytes(w0)
+    n_copies = n_rotating_copies(logit_bytes)
+    sets, host_first = make_sets(w_rank, n_copies, dev, ssd, synth)
 
-    # outcome statistics from the last step of each rotating copy
-    r0 = outs[0]
-    n_acc = r0.n_accepted.cpu().numpy()
-    hit = r0.hit.cpu().numpy()
-    st = r0.status.cpu().numpy()
+    points = [dict()]
+    if args.sweep:
+        points = [dict(T=T, fanout_mode=m, C=C, alpha=synth.SWEEP_ALPHA[T])
+                  for T in (0.0, 0.6, 1.0) for m in (0, 1) for C in (1.0, 0.5, 0.2)]
+    results = []
+    for pt in points:
+        w = w_rank.replace(**pt)
+        draw_tokens(w, sets, dev, ssd)
+        ws = ssd.Workspace(w.B, w.K, dev, w.V, ssd.DTYPE_BF16 if w.dtype == "bf16" else ssd.DTYPE_FP32)
+        outs = [ssd.alloc_verify_result(w.B, w.K, w.budget, dev, True) for _ in range(n_copies)]
 
-    result = dict(rows_per_s=rows_per_s, ms_per_step=ms_per_step, kernel_ms=kernel_ms, clocks=clocks,
-                  launches=steps_done * KERNELS_PER_VERIFY, mean_accepted=float(n_acc.mean()), hit_rate=float(hit.mean()),
-                  near_tie_rows=int(((st & ssd.ROW_NEAR_TIE) != 0).sum()), n_copies=n_copies,
-                  alg_bytes=alg_bytes, logit_bytes=logit_bytes)
-
-    # End to end through the public API from pinned host buffers (rank 0, N=1 only).
-    if rank == 0 and world == 1 and not args.no_e2e:
-        ht = torch.from_numpy(host_first["target"].view(np.int16)).view(torch.bfloat16).pin_memory() \
-            if host_first["target"].dtype == np.uint16 else torch.from_numpy(host_first["target"]).pin_memory()
-        hd = torch.from_numpy(host_first["draft"].view(np.int16)).view(torch.bfloat16).pin_memory() \
-            if host_first["draft"].dtype == np.uint16 else torch.from_numpy(host_first["draft"]).pin_memory()
-        htok = sets[0]["tok"].cpu().pin_memory()
-        hu = torch.from_numpy(host_first["uniforms"]).pin_memory()
-        ha = torch.from_numpy(host_first["alpha"]).pin_memory()
-        h2d = sum(x.numel() * x.element_size() for x in (ht, hd, htok, hu, ha))
-        probe = ssd.ssd_verify_host(ht, hd, htok, hu, w.T, ha, w.budget, w.C, dev,
-                                    fallback_seed=w_rank.fallback_seed, workspace=ws)
-        d2h = sum(v.numel() * v.element_size() for v in probe.__dict__.values() if isinstance(v, torch.Tensor))
-        e_steps = max(3, min(args.steps, 10))
+        if args.unfused:
+            def step(i, w=w, ws=ws, outs=outs):
+                # the five calls of the unfused step on one stream
+                s = sets[i % n_copies]
+                o = outs[i % n_copies]
+                F = ssd.ssd_fanout_plan(s["alpha"], w.K, w.budget, w.fanout_mode, F=s["F"])
+                rw = ssd.ssd_saguaro_reweight(s["d"], w.T, F, w.C, w.budget, guess=s["t"][:, w.K, :],
+                                              guess_row_stride=(w.K + 1) * w.V, workspace=ws)
+                ver = ssd.ssd_verify(s["t"], s["d"], s["tok"], s["u"], w.T, F=F, C_coef=w.C, budget=w.budget,
+                                     cache=False, workspace=ws, out=o)
+                offs, toks = ssd.ssd_cache_build(F, rw.topf_tokens, w.budget)
+                hit, slot, nxt = ssd.ssd_cache_lookup(offs, toks, ver.n_accepted, ver.bonus, w.V,
+                                                      fallback_seed=w.fallback_seed)
+                o.hit, o.slot, o.next_tokens = hit, slot, nxt
+            kernels = KERNELS_PER_UNFUSED
+        else:
+            def step(i, w=w, ws=ws, outs=outs):
+                # one launch pair: the fan-out plan is computed inside the fused kernel from alpha
+                s = sets[i % n_copies]
+                ssd.ssd_verify(s["t"], s["d"], s["tok"], s["u"], w.T, alpha=s["alpha"], fanout_mode=w.fanout_mode,
+                               C_coef=w.C, budget=w.budget, cache=True, fallback_seed=w.fallback_seed,
+                               workspace=ws, out=outs[i % n_copies])
+            kernels = KERNELS_PER_VERIFY
+        total_ms, per_step, clocks = time_steps(step, args.steps, args.warmup, dev, world, dist,
+                                                local_rank if rank == 0 else None)
+        if world > 1:
+            total_ms = max_over_ranks(total_ms, dist, dev)
+        # outcome statistics over every rotating copy's last step
         torch.cuda.synchronize()
-        t0 = torch.cuda.Event(enable_timing=True)
-        t1 = torch.cuda.Event(enable_timing=True)
-        t0.record(stream)
-        for _ in range(e_steps):
-            ssd.ssd_verify_host(ht, hd, htok, hu, w.T, ha, w.budget, w.C, dev, fallback_seed=w_rank.fallback_seed,
-                                workspace=ws)
-        t1.record(stream)
-        torch.cuda.synchronize()
-        e_ms = t0.elapsed_time(t1) / e_steps
-        result["e2e"] = {"value": w.B / (e_ms / 1e3), "unit": "rows/s", "h2d_bytes_per_step": int(h2d),
-                         "d2h_bytes_per_step": int(d2h), "ms_per_step": e_ms}
-    return result
+        n_acc = np.concatenate([o.n_accepted.cpu().numpy() for o in outs])
+        hit = np.concatenate([o.hit.cpu().numpy() for o in outs])
+        st = np.concatenate([o.status.cpu().numpy() for o in outs])
+        res = dict(point=pt, w=w, rows_per_s=job_rows_per_s(world, w.B, args.steps, total_ms),
+                   ms_per_step=total_ms / args.steps, per_step_ms=per_step, clocks=clocks,
+                   launches=args.steps * kernels, mean_accepted=float(n_acc.mean()), hit_rate=float(hit.mean()),
+                   near_tie_rows=int(((st & ssd.ROW_NEAR_TIE) != 0).sum()), n_copies=n_copies, alg_bytes=alg_bytes,
+                   logit_bytes=logit_bytes)
+
+        # End to end through the public API from pinned host buffers (rank 0,
+        # N=1, default fused step only).
+        if rank == 0 and world == 1 and not args.no_e2e and not args.unfused and not args.sweep:
+            def pin(x):
+                if x.dtype == np.uint16:
+                    return torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).pin_memory()
+                return torch.from_numpy(x).pin_memory()
+            ht, hd = pin(host_first["target"]), pin(host_first["draft"])
+            htok = sets[0]["tok"].cpu().pin_memory()
+            hu = torch.from_numpy(host_first["uniforms"]).pin_memory()
+            ha = torch.full((w.B,), w.alpha, dtype=torch.float32).pin_memory()
+            h2d = sum(x.numel() * x.element_size() for x in (ht, hd, htok, hu, ha))
+            probe = ssd.ssd_verify_host(ht, hd, htok, hu, w.T, ha, w.budget, w.C, dev,
+                                        fallback_seed=w.fallback_seed, workspace=ws)
+            d2h = sum(v.numel() * v.element_size() for v in probe.__dict__.values() if isinstance(v, torch.Tensor))
+            e_steps = max(3, min(args.steps, 10))
+            stream = torch.cuda.current_stream(dev)
+            torch.cuda.synchronize()
+            t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            t0.record(stream)
+            for _ in range(e_steps):
+                ssd.ssd_verify_host(ht, hd, htok, hu, w.T, ha, w.budget, w.C, dev, fallback_seed=w.fallback_seed,
+                                    workspace=ws)
+            t1.record(stream)
+            torch.cuda.synchronize()
+            e_ms = t0.elapsed_time(t1) / e_steps
+            res["e2e"] = {"value": w.B / (e_ms / 1e3), "unit": "rows/s", "h2d_bytes_per_step": int(h2d),
+                          "d2h_bytes_per_step": int(d2h), "ms_per_step": e_ms}
+        results.append(res)
+        del ws, outs
+    return results
 
 
 def cpu_baseline(w, seconds_target=15.0, reference_rows=None):
@@ -361,14 +413,64 @@ def run_reference(args, rank, world):
     print(json.dumps(line), flush=True)
 
 
+def build_line(args, res, world):
+    w = res["w"]
+    peak, peak_kind = measured_peaks()
+    per = res["per_step_ms"]
+    k_avg = sum(per) / len(per)   # average launch duration over the timed region
+    achieved = res["alg_bytes"] / (k_avg / 1e3) / 1e9
+    traffic = recorded_traffic(w.name) if not args.unfused and not args.sweep else None
+    cfg = dict(workload_config(w, world),
+               l2=f"{res['n_copies']} rotating input copies of {res['logit_bytes'] / 1e6:.1f} MB "
+                  f"(together > 2 x 126 MB L2)")
+    if args.unfused:
+        cfg["step"] = "unfused: fan-out plan, reweight, verify, cache build, cache lookup (one stream)"
+    line = {
+        "metric": METRIC,
+        "value": res["rows_per_s"],
+        "unit": "rows/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": res["ms_per_step"],
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": w.dtype,
+        "data": "synthetic",
+        "config": cfg,
+        "hbm_gbs": achieved,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "traffic": traffic,
+                     "kernel": ssd_step_kernels() if not args.unfused else "the five-call step, timed as a whole",
+                     "peak_source": f"{peak_kind} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)"
+                     if peak_kind == "measured" else "fallback 6650 GB/s",
+                     "kernel_us_avg": k_avg * 1e3, "kernel_us_min": min(per) * 1e3,
+                     "alg_bytes_per_launch": res["alg_bytes"]},
+        "gpu_launches": res["launches"],
+        "mean_accepted": res["mean_accepted"],
+        "hit_rate": res["hit_rate"],
+        "miss_rate": 1.0 - res["hit_rate"],
+        "near_tie_rows": res["near_tie_rows"],
+    }
+    if res.get("clocks"):
+        line["clocks"] = res["clocks"]
+    if "e2e" in res:
+        line["e2e"] = res["e2e"]
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w, seconds_target=5.0 if args.sweep else 15.0)
+    return line
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--repeat", type=int, default=4, help="timed replays of the graph of --steps launches")
     ap.add_argument("--impl", default="ssd", choices=["ssd", "reference"])
     ap.add_argument("--workload", default=None)
+    ap.add_argument("--sweep", action="store_true", help="temperature x fan-out mode x C grid, one line each")
+    ap.add_argument("--unfused", action="store_true", help="time the five-call unfused step")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
@@ -376,6 +478,7 @@ def main():
     if args.workload is None:
         args.workload = synth.HEADLINE
     args.warmup = max(args.warmup, 3)
+    args.steps = max(args.steps, 1)
 
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -394,55 +497,15 @@ def main():
         torch.cuda.set_device(local_rank)
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local_rank))
-    res = run_ssd(args, rank, world, local_rank)
+    results = run_ssd(args, rank, world, local_rank)
     if world > 1:
         import torch.distributed as dist
         dist.barrier()
         dist.destroy_process_group()
     if rank != 0:
         return
-    w = synth.WORKLOADS[args.workload]
-    peak, peak_kind = measured_peaks()
-    kms = sorted(res["kernel_ms"])
-    k_avg = sum(kms) / len(kms)   # average launch duration over the timed region
-    achieved = res["alg_bytes"] / (k_avg / 1e3) / 1e9
-    traffic = recorded_traffic(w.name)
-    line = {
-        "metric": METRIC,
-        "value": res["rows_per_s"],
-        "unit": "rows/s",
-        "n_gpus": world,
-        "steps": args.steps * max(1, args.repeat),
-        "warmup": args.warmup,
-        "ms_per_step": res["ms_per_step"],
-        "higher_is_better": True,
-        "scaling": "weak",
-        "vs_baseline": None,
-        "dtype": w.dtype,
-        "data": "synthetic",
-        "config": dict(workload_config(w, world),
-                       l2=f"{res['n_copies']} rotating input copies of {res['logit_bytes'] / 1e6:.1f} MB "
-                          f"(each > 126 MB L2)"),
-        "hbm_gbs": achieved,
-        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                     "frac": achieved / peak, "traffic": traffic,
-                     "kernel": ssd_step_kernels(),
-                     "peak_source": f"{peak_kind} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)"
-                     if peak_kind == "measured" else "fallback 6650 GB/s",
-                     "kernel_us_avg": k_avg * 1e3, "kernel_us_min": kms[0] * 1e3,
-                     "alg_bytes_per_launch": res["alg_bytes"]},
-        "gpu_launches": res["launches"],
-        "mean_accepted": res["mean_accepted"],
-        "hit_rate": res["hit_rate"],
-        "near_tie_rows": res["near_tie_rows"],
-    }
-    if res.get("clocks"):
-        line["clocks"] = res["clocks"]
-    if "e2e" in res:
-        line["e2e"] = res["e2e"]
-    if world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(w)
-    print(json.dumps(line), flush=True)
+    for res in results:
+        print(json.dumps(build_line(args, res, world)), flush=True)
 
 
 if __name__ == "__main__":

@@ -34,5 +34,19 @@ def build(force: bool = False, verbose: bool = False) -> str:
     return LIB
 
 
+def build_variant(name: str, defines, force: bool = False) -> str:
+    """A build of the same sources with extra -D flags (test builds, e.g. a
+    short dependency-wait limit), next to libssd.so as libssd_<name>.so."""
+    out = os.path.join(HERE, f"libssd_{name}.so")
+    if not force and os.path.exists(out) and all(os.path.getmtime(out) >= os.path.getmtime(d) for d in DEPS):
+        return out
+    cmd = [nvcc()] + NVCC_FLAGS + [f"-D{d}" for d in defines] + SOURCES + ["-o", out + ".tmp"]
+    res = subprocess.run(cmd, capture_output=True, text=True)
+    if res.returncode != 0:
+        raise RuntimeError("nvcc failed:\n" + res.stdout + res.stderr)
+    os.replace(out + ".tmp", out)
+    return out
+
+
 if __name__ == "__main__":
     build(force=True, verbose=True)

@@ -63,7 +63,12 @@ constexpr int kSelCap = 512;           // >= SSD_MAX_BUDGET
 constexpr int kMaxGroups = kThreads;   // thread maxima per CTA
 constexpr unsigned long long kRingWaitNs = 2000000000ull;  // a ring stage's bytes: 2 s at most
 constexpr float kNearTie = 1e-5f;
-constexpr unsigned long long kDepWaitNs = 1000000000ull;  // a draw's wait for its row decision
+#ifndef SSD_DEP_WAIT_NS
+#define SSD_DEP_WAIT_NS 1000000000ull
+#endif
+// the limit of a wait for another CTA's result (a slice partial, a unit record,
+// a row's decision word): 1 s
+constexpr unsigned long long kDepWaitNs = SSD_DEP_WAIT_NS;
 constexpr int kFlagTimeout = SSD_ROW_DEVICE_TIMEOUT;
 constexpr size_t kRingBytes = static_cast<size_t>(kStages) * 2 * kChunkVecs * 16;
 
@@ -162,6 +167,11 @@ struct Args {
   uint32_t* epoch;         // calls completed on this workspace (kernel 2 advances it)
   int32_t* k2_done;        // kernel 2 CTAs past their wait
   int32_t* error;
+  // the persistent fused verify kernel
+  int32_t* queue;          // next work item
+  int32_t* fdone;          // CTAs finished
+  int lag;                 // rows between a row's statistics items and its draw items
+  int n_items;
 };
 
 template <typename TIn>
@@ -292,27 +302,38 @@ __device__ __forceinline__ void merge_ms(float& m, float& s, float m2, float s2,
   s = a + b;
 }
 
-// Exact top-F of a whole row, read from global memory by one CTA: a radix
+// The CTA barrier, and the barrier of the 256 consumer threads of a kernel
+// whose last warp only issues copies (named barrier 1).
+struct CtaBarrier {
+  __device__ __forceinline__ void operator()() const { __syncthreads(); }
+};
+struct ConsumerBarrier {
+  __device__ __forceinline__ void operator()() const { asm volatile("bar.sync 1, 256;" ::: "memory"); }
+};
+
+// Exact top-F of a whole row, read from global memory by 256 threads: a radix
 // select on the 32-bit order key (four 8-bit digits), ties at the threshold
 // taken in token-id order, then the F winners ranked by (key, id) in place.
 // Used when the shared-memory candidate filter cannot bound the set (many
-// ties, F large).  `hist` needs 256 ints; the result is sel[0 .. F).
-template <typename TIn>
-__device__ void topf_exact_global(const TIn* row, int V, int F, Cand* sel, int32_t* hist, int tid) {
+// ties, F large).  `hist` needs 256 ints; the result is sel[0 .. F); `bar`
+// synchronises the 256 threads.
+
+template <typename TIn, typename Bar>
+__device__ void topf_exact_global(const TIn* row, int V, int F, Cand* sel, int32_t* hist, int tid, Bar bar) {
   __shared__ uint32_t s_prefix, s_mask;
   __shared__ int32_t s_remaining, s_napp, s_tie_base[kThreads + 1];
   if (tid == 0) { s_prefix = 0u; s_mask = 0u; s_remaining = F; s_napp = 0; }
-  __syncthreads();
+  bar();
   for (int level = 0; level < 4; ++level) {
     const int shift = 24 - 8 * level;
     for (int i = tid; i < 256; i += kThreads) hist[i] = 0;
-    __syncthreads();
+    bar();
     const uint32_t prefix = s_prefix, mask = s_mask;
     for (int v = tid; v < V; v += kThreads) {
       const uint32_t k = ord_key(Elem<TIn>::at(row, v));
       if ((k & mask) == prefix) atomicAdd(&hist[(k >> shift) & 255u], 1);
     }
-    __syncthreads();
+    bar();
     if (tid == 0) {
       int cum = 0, rem = s_remaining, d = 255;
       for (; d > 0; --d) {
@@ -323,7 +344,7 @@ __device__ void topf_exact_global(const TIn* row, int V, int F, Cand* sel, int32
       s_prefix = prefix | (static_cast<uint32_t>(d) << shift);
       s_mask = mask | (255u << shift);
     }
-    __syncthreads();
+    bar();
   }
   const uint32_t t = s_prefix;
   const int need_eq = s_remaining;
@@ -333,12 +354,12 @@ __device__ void topf_exact_global(const TIn* row, int V, int F, Cand* sel, int32
   int my_eq = 0;
   for (int v = lo; v < hi; ++v) my_eq += (ord_key(Elem<TIn>::at(row, v)) == t);
   s_tie_base[tid + 1] = my_eq;
-  __syncthreads();
+  bar();
   if (tid == 0) {
     s_tie_base[0] = 0;
     for (int i = 1; i <= kThreads; ++i) s_tie_base[i] += s_tie_base[i - 1];
   }
-  __syncthreads();
+  bar();
   int tie_rank = s_tie_base[tid];
   for (int v = lo; v < hi; ++v) {
     const float x = Elem<TIn>::at(row, v);
@@ -354,7 +375,7 @@ __device__ void topf_exact_global(const TIn* row, int V, int F, Cand* sel, int32
       ++tie_rank;
     }
   }
-  __syncthreads();
+  bar();
   // Rank in place: every thread keeps its (at most two) winners in registers.
   constexpr int kPer = kSelCap / kThreads;
   Cand mine[kPer];
@@ -371,11 +392,11 @@ __device__ void topf_exact_global(const TIn* row, int V, int F, Cand* sel, int32
       rk[q] = r;
     }
   }
-  __syncthreads();
+  bar();
 #pragma unroll
   for (int q = 0; q < kPer; ++q)
     if (rk[q] >= 0) sel[rk[q]] = mine[q];
-  __syncthreads();
+  bar();
 }
 
 // Fan-out plan of one row ([ZH] section 2 challenge 1; [NL] section 3A):
@@ -1108,7 +1129,7 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) ssd_stats_kernel(const _
   }
   if (slow) {
     const TIn* row = srcQ ? baseQ + rbQ : baseP + rbP;
-    topf_exact_global<TIn>(row, V, Fj, sel, sm.hist, tid);
+    topf_exact_global<TIn>(row, V, Fj, sel, sm.hist, tid, CtaBarrier{});
   }
   __syncthreads();
 
