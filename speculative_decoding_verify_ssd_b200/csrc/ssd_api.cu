@@ -526,7 +526,7 @@ ssd_status ssd_verify(const void* target_logits, const void* draft_logits, const
     a.chunk = fp.chunk;
     return launch_fused(a, dtype, static_cast<cudaStream_t>(stream));
   }
-  return launch(a, dtype, false, units, B, static_cast<cudaStream_t>(stream));
+  return launch(a, dtype, V % VE == 0, units, B, static_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"
