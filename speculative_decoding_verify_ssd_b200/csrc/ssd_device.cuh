@@ -105,6 +105,20 @@ __device__ __forceinline__ int32_t arrive_acq_rel_gpu(int32_t* p) {
 }
 
 
+// CTA-scope acquire-release add on a shared-memory counter; returns the old value.
+__device__ __forceinline__ uint32_t atom_add_acq_rel_cta_shared(uint32_t* p, uint32_t v) {
+  uint32_t old;
+  asm volatile("atom.acq_rel.cta.shared::cta.add.u32 %0, [%1], %2;" : "=r"(old) : "r"(smem_addr(p)), "r"(v) : "memory");
+  return old;
+}
+
+// Orders this thread's view of generic-proxy shared-memory accesses (the
+// other warps' reads of a stage, acquired above) before its later
+// async-proxy ones (the bulk copy that overwrites the stage).
+__device__ __forceinline__ void fence_proxy_async_shared() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 __device__ __forceinline__ uint64_t ld_acquire_gpu_u64(const uint64_t* p) {
   uint64_t v;
   asm volatile("ld.acquire.gpu.global.b64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");

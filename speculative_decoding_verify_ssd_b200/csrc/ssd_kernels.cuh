@@ -70,6 +70,9 @@ constexpr float kNearTie = 1e-5f;
 // a row's decision word): 1 s
 constexpr unsigned long long kDepWaitNs = SSD_DEP_WAIT_NS;
 constexpr int kFlagTimeout = SSD_ROW_DEVICE_TIMEOUT;
+#ifndef SSD_LAST_ARRIVES
+#define SSD_LAST_ARRIVES 1  // the last slice / unit to arrive finalises (no waits)
+#endif
 constexpr size_t kRingBytes = static_cast<size_t>(kStages) * 2 * kChunkVecs * 16;
 
 static_assert(8 * (kCandCap + kGatherCap + kSelCap) <= kRingBytes, "merge buffers must fit in the idle ring");
@@ -513,14 +516,22 @@ __device__ __forceinline__ void fanout_row_power(float alpha_f, int K, int budge
   }
 }
 
+#ifndef SSD_RING_WARP_RELEASE
+#define SSD_RING_WARP_RELEASE 1
+#endif
+
 // Ring of bulk copies that streams one slice of up to two rows of a unit
 // through shared memory, chunk by chunk (CV 16-byte vectors per row per
-// chunk, ST stages).  Thread 0 issues and polls; the other threads sleep in the
-// CTA barrier and then take one acquiring look at the stage's phase.
+// chunk, ST stages).  Every thread waits on the chunk's full barrier itself;
+// after reading a stage, each warp counts its release on the stage's counter,
+// and the warp that completes the count refills the stage with the chunk ST
+// ahead.  No CTA barrier sits in the stream, and no warp waits for the
+// slowest one except through the data it needs.
 template <typename TIn, int CV = kChunkVecs, int ST = kStages>
 struct Ring {
   unsigned char* buf;
   uint64_t* full;
+  uint32_t* rel;  // [ST] warps done with the stage's current chunk
   const TIn* row0;
   const TIn* row1;
   int nrows, e0, nvec, nch, n_issued;
@@ -541,13 +552,40 @@ struct Ring {
   __device__ __forceinline__ void start(int tid) {
     n_issued = 0;
     if (tid == 0) {
-      for (int s = 0; s < ST; ++s) mbar_init(&full[s], 1);
+      for (int s = 0; s < ST; ++s) {
+        mbar_init(&full[s], 1);
+        rel[s] = 0u;
+      }
       mbar_init_fence();
     }
     __syncthreads();
     if (tid == 0)
       for (int c = 0; c < min(ST, nch); ++c) issue(c);
   }
+#if SSD_RING_WARP_RELEASE
+  // Chunk c is ready for this thread.
+  __device__ __forceinline__ void acquire(int c, int tid, int& tmo) {
+    if (!mbar_wait_bounded(&full[c % ST], (c / ST) & 1, kRingWaitNs)) tmo = 1;
+  }
+  // This warp is done with chunk c's stage; the last warp to say so refills it.
+  __device__ __forceinline__ void release(int c, int lane) {
+    __syncwarp();
+    if (lane == 0) {
+      const int slot = c % ST;
+      if (atom_add_acq_rel_cta_shared(&rel[slot], 1u) == static_cast<uint32_t>(kWarps - 1)) {
+        rel[slot] = 0u;
+        fence_proxy_async_shared();
+        if (c + ST < nch) issue(c + ST);
+      }
+    }
+  }
+  // Never leave a copy in flight (only a timed-out wait can leave one): every
+  // chunk is issued by the time all are released; wait for the last ST.
+  __device__ __forceinline__ void drain(int tid, int tmo) {
+    if (tmo && tid == 0)
+      for (int c = max(0, nch - ST); c < nch; ++c) mbar_wait_bounded(&full[c % ST], (c / ST) & 1, kRingWaitNs);
+  }
+#else
   // Chunk c is ready for every thread; the barrier also marks chunk c - 1
   // consumed, so its stage is refilled.
   __device__ __forceinline__ void acquire(int c, int tid, int& tmo) {
@@ -556,14 +594,15 @@ struct Ring {
     if (tid == 0 && c > 0 && c - 1 + ST < nch) issue(c - 1 + ST);
     if (tid != 0 && !mbar_try_wait(&full[c % ST], (c / ST) & 1, 0u)) tmo = 1;
   }
-  __device__ __forceinline__ uint4 vec(int c, int r, int tid) const {
-    return *reinterpret_cast<const uint4*>(stage(c % ST, r) + tid * 16);
-  }
-  // Never leave a copy in flight (only a timed-out wait can leave one).
+  __device__ __forceinline__ void release(int, int) {}
   __device__ __forceinline__ void drain(int tid, int tmo) {
     if (tmo && tid == 0)
       for (int c = max(0, n_issued - ST); c < n_issued; ++c)
         mbar_wait_bounded(&full[c % ST], (c / ST) & 1, kRingWaitNs);
+  }
+#endif
+  __device__ __forceinline__ uint4 vec(int c, int r, int tid) const {
+    return *reinterpret_cast<const uint4*>(stage(c % ST, r) + tid * 16);
   }
 };
 
@@ -679,6 +718,7 @@ __device__ __forceinline__ void load_plan(const Args& a, int b, int32_t* s_F, in
 // Shared memory of kernel 1.
 struct Smem1 {
   uint64_t full[kStages];
+  uint32_t rel[kStages];
   float wred[kWarps][4];
   int32_t wint[kWarps][2];
   float gmax[kMaxGroups];
@@ -728,6 +768,7 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) ssd_stats_kernel(const _
   Ring<TIn, kStatsChunkVecs, kStatsStages> ring;
   ring.buf = ring_buf;
   ring.full = sm.full;
+  ring.rel = sm.rel;
   ring.row0 = hasP ? baseP + rbP : baseQ + rbQ;
   ring.row1 = baseQ + rbQ;
   ring.nrows = (hasP ? 1 : 0) + (hasQ ? 1 : 0);
@@ -849,6 +890,7 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) ssd_stats_kernel(const _
       }
     }
     }
+    if constexpr (kAligned) ring.release(c, lane);
   }
   if constexpr (kGreedy) {
     if (nan_seen) { mP = __int_as_float(0x7FC00000); mQ = mP; }
@@ -1016,6 +1058,14 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) ssd_stats_kernel(const _
   }
   __syncthreads();
   if constexpr (kAligned) ring.drain(tid, tmo);
+#if SSD_LAST_ARRIVES
+  // The unit's last slice to arrive finalizes; the others leave.  Nobody
+  // waits: the arrival is one acquire-release reduction per slice.
+  if (tid == 0) sm.is_last = arrive_acq_rel_gpu(a.arrive1 + u) == S - 1 ? 1 : 0;
+  __syncthreads();
+  if (!sm.is_last) return;
+  const bool arrivals_ok = true;
+#else
   // The unit's last slice, the last of its CTAs to be scheduled, finalizes:
   // the others publish and leave without waiting; it waits (bounded) until
   // they have all published.
@@ -1029,6 +1079,7 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) ssd_stats_kernel(const _
   }
   __syncthreads();
   const bool arrivals_ok = sm.is_last != 0;
+#endif
 
   // =============== the unit's finalizer: its last slice, once all have arrived ======
   const SlicePart* parts = a.parts + u * S;
@@ -1206,6 +1257,13 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) ssd_stats_kernel(const _
     a.arrive1[u] = 0;
   }
   __syncthreads();
+#if SSD_LAST_ARRIVES
+  // Likewise per row: the last unit of the row to arrive decides.
+  if (tid == 0) sm.is_last_row = arrive_acq_rel_gpu(a.row_arrive + b) == upr - 1 ? 1 : 0;
+  __syncthreads();
+  if (!sm.is_last_row) return;
+  const bool row_ok = true;
+#else
   // Likewise per row: unit j = 0, whose CTAs are the row's last to be
   // scheduled, decides once the other units have published.
   if (j != 0) {
@@ -1218,6 +1276,7 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) ssd_stats_kernel(const _
   }
   __syncthreads();
   const bool row_ok = sm.is_last_row != 0;
+#endif
 
   // =============== the row's decision: unit j = 0, once all units have arrived ======
   // One warp; lane k reads unit k's record (k = 32 only when K = 32), so the
@@ -1296,6 +1355,7 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) ssd_stats_kernel(const _
 // Shared memory of kernel 2.
 struct Smem2 {
   uint64_t full[kStages];
+  uint32_t rel[kStages];
   int32_t dep_ok, w_kstar, w_flags;
   float rs[kMaxChunks][kWarps];
   float ps[kMaxChunks][kWarps];
@@ -1421,6 +1481,7 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) ssd_draw_kernel(const __
   Ring<TIn> ring;
   ring.buf = ring_buf;
   ring.full = sm.full;
+  ring.rel = sm.rel;
   ring.row0 = useP ? baseP + rbP : baseQ + rbQ;
   ring.row1 = useQ ? baseQ + rbQ : nullptr;
   ring.nrows = (useP ? 1 : 0) + (useQ ? 1 : 0);
@@ -1473,6 +1534,7 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) ssd_draw_kernel(const __
       rsum = warp_sum(rsum);
       psum = warp_sum(psum);
       if (lane == 0) { sm.rs[c][warp] = rsum; sm.ps[c][warp] = psum; }
+      if constexpr (kAligned) ring.release(c, lane);
     }
     tmo = __syncthreads_or(tmo);
     if (warp == 0) {  // the slice's masses: lane l sums entries l, l + 32, ... then a butterfly
