@@ -13,7 +13,6 @@
 #include "../../include/ssd.h"
 #include "ssd_device.cuh"
 #include "ssd_kernels.cuh"
-#include "ssd_fused.cuh"
 
 namespace ssd {
 
@@ -203,30 +202,9 @@ static cudaError_t prepare_kernel(const void* fn) {
 // counters (zero between calls) and the error word.
 struct WsLayout {
   size_t parts, ustate, dparts, rstate, arrive1, row_arrive, draw_arrive, row_arrive2, rflag, epoch, k2_done, error,
-      queue, fdone, total;
+      total;
   int n_slices;
 };
-
-#ifndef SSD_ITEM_BYTES
-#define SSD_ITEM_BYTES 131072  // logits per statistics item of the fused kernel (both rows of a unit slice)
-#endif
-constexpr long long kItemBytes = SSD_ITEM_BYTES;
-
-// Slices of a unit for the fused kernel's statistics items: about
-// kItemBytes of logits per item, at most kMaxSlices.
-static Plan fused_plan(int V, int esize) {
-  const int VE = 16 / esize;
-  long long ns = (2LL * V * esize + kItemBytes - 1) / kItemBytes;
-  if (ns > kMaxSlices) ns = kMaxSlices;
-  if (ns < 1) ns = 1;
-  long long chunk = (V + ns - 1) / ns;
-  chunk = (chunk + VE - 1) / VE * VE;
-  ns = (V + chunk - 1) / chunk;
-  Plan p;
-  p.n_slices = static_cast<int>(ns);
-  p.chunk = static_cast<int>(chunk);
-  return p;
-}
 
 static int plan_slices(int B, int K, int V, int dtype) {
   const int esize = dtype == SSD_DTYPE_FP32 ? 4 : 2;
@@ -238,8 +216,6 @@ static int plan_slices(int B, int K, int V, int dtype) {
   if (make_plan(V, 2, esize, B, &p2, kDrawCtaBytes) == SSD_OK) ns = ns > p2.n_slices ? ns : p2.n_slices;
   if (make_plan(V, 1, esize, static_cast<long long>(B) * K, &p1, kDrawCtaBytes) == SSD_OK)
     ns = ns > p1.n_slices ? ns : p1.n_slices;
-  const Plan pf = fused_plan(V, esize);
-  ns = ns > pf.n_slices ? ns : pf.n_slices;
   return ns;
 }
 
@@ -264,8 +240,6 @@ static WsLayout ws_layout(int B, int K, int V, int dtype) {
   w.epoch = off;       off += sizeof(uint32_t);
   w.k2_done = off;     off += sizeof(int32_t);
   w.error = off;       off += sizeof(int32_t);
-  w.queue = off;       off += sizeof(int32_t);
-  w.fdone = off;       off += sizeof(int32_t);
   w.total = up256(off);
   return w;
 }
@@ -284,8 +258,6 @@ static void bind_workspace(Args& a, void* ws, const WsLayout& w) {
   a.epoch = reinterpret_cast<uint32_t*>(base + w.epoch);
   a.k2_done = reinterpret_cast<int32_t*>(base + w.k2_done);
   a.error = reinterpret_cast<int32_t*>(base + w.error);
-  a.queue = reinterpret_cast<int32_t*>(base + w.queue);
-  a.fdone = reinterpret_cast<int32_t*>(base + w.fdone);
 }
 
 template <typename TIn, bool kAligned, bool kGreedy>
@@ -333,57 +305,6 @@ static ssd_status launch(const Args& a, int dtype, bool aligned, long long units
 }
 
 static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
-
-// The persistent fused verify kernel: one CTA per resident slot (at most one
-// per work item), the queue order's lag from the bytes in flight.
-template <typename TIn, bool kGreedy>
-static ssd_status launch_fused_t(Args a, cudaStream_t stream) {
-  const void* fn = reinterpret_cast<const void*>(&ssd_fused_kernel<TIn, kGreedy>);
-  static std::mutex mu;
-  static std::map<int, int> occ_by_dev;
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return SSD_ERR_CUDA;
-  int occ = 0;
-  {
-    std::lock_guard<std::mutex> lock(mu);
-    auto it = occ_by_dev.find(dev);
-    if (it == occ_by_dev.end()) {
-      if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kFusedRingBytes)) !=
-          cudaSuccess)
-        return SSD_ERR_CUDA;
-      if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, fn, kFusedThreads, kFusedRingBytes) != cudaSuccess)
-        return SSD_ERR_CUDA;
-      occ_by_dev[dev] = occ;
-    } else {
-      occ = it->second;
-    }
-  }
-  if (occ < 1) return SSD_ERR_UNSUPPORTED;
-  const long long slots = static_cast<long long>(occ) * sm_count();
-  const int esize = static_cast<int>(sizeof(TIn));
-  const long long row_bytes = static_cast<long long>(2 * a.K + 1) * a.V * esize;
-  const long long item_bytes = 2LL * a.chunk * esize;
-#ifndef SSD_LAG_MULT
-#define SSD_LAG_MULT 4  // rows of lag per row of work in flight
-#endif
-  long long lag = SSD_LAG_MULT * ((slots * item_bytes + row_bytes - 1) / row_bytes) + 1;
-  if (lag > a.B) lag = a.B;
-  if (lag < 1) lag = 1;
-  a.lag = static_cast<int>(lag);
-  const long long n_items = static_cast<long long>(a.B) * (a.units_per_row * a.n_slices + a.d_slices);
-  if (n_items > 0x7FFFFFFFLL) return SSD_ERR_INVALID_ARG;
-  a.n_items = static_cast<int>(n_items);
-  const long long grid = n_items < slots ? n_items : slots;
-  ssd_fused_kernel<TIn, kGreedy><<<static_cast<unsigned>(grid), kFusedThreads, kFusedRingBytes, stream>>>(a);
-  return cudaGetLastError() == cudaSuccess ? SSD_OK : SSD_ERR_CUDA;
-}
-
-static ssd_status launch_fused(const Args& a, int dtype, cudaStream_t stream) {
-  const bool greedy = a.T == 0.f;
-  if (dtype == SSD_DTYPE_BF16)
-    return greedy ? launch_fused_t<uint16_t, true>(a, stream) : launch_fused_t<uint16_t, false>(a, stream);
-  return greedy ? launch_fused_t<float, true>(a, stream) : launch_fused_t<float, false>(a, stream);
-}
 
 }  // namespace ssd
 
@@ -514,18 +435,6 @@ ssd_status ssd_verify(const void* target_logits, const void* draft_logits, const
   }
   bind_workspace(a, workspace, wl);
   const int VE = 16 / esize;
-#ifndef SSD_USE_FUSED
-#define SSD_USE_FUSED 0
-#endif
-  if (SSD_USE_FUSED && V % VE == 0) {
-    // rows start on 16-byte boundaries: the persistent fused kernel, with its
-    // own statistics slices
-    const Plan fp = fused_plan(V, esize);
-    if (fp.n_slices > wl.n_slices) return SSD_ERR_WORKSPACE;
-    a.n_slices = fp.n_slices;
-    a.chunk = fp.chunk;
-    return launch_fused(a, dtype, static_cast<cudaStream_t>(stream));
-  }
   return launch(a, dtype, V % VE == 0, units, B, static_cast<cudaStream_t>(stream));
 }
 

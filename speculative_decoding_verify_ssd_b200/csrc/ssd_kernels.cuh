@@ -170,11 +170,6 @@ struct Args {
   uint32_t* epoch;         // calls completed on this workspace (kernel 2 advances it)
   int32_t* k2_done;        // kernel 2 CTAs past their wait
   int32_t* error;
-  // the persistent fused verify kernel
-  int32_t* queue;          // next work item
-  int32_t* fdone;          // CTAs finished
-  int lag;                 // rows between a row's statistics items and its draw items
-  int n_items;
 };
 
 template <typename TIn>
@@ -732,22 +727,16 @@ struct Smem1 {
   int32_t cnt[kMaxSlices];
 };
 
+// One statistics CTA: slice `slice` of unit (row b, position j).
 template <typename TIn, bool kAligned, bool kGreedy>
-__global__ void __launch_bounds__(kThreads, kMinBlocks) ssd_stats_kernel(const __grid_constant__ Args a) {
+__device__ __forceinline__ void stats_cta(const Args& a, int b, int j, int slice) {
   constexpr int VE = Elem<TIn>::VE;
   extern __shared__ __align__(128) unsigned char ring_buf[];
   __shared__ __align__(16) Smem1 sm;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int S = a.n_slices;
-  const int order = blockIdx.x / S, slice = blockIdx.x % S;
   const int upr = a.units_per_row;
-  // rows in order, so that rows are decided (and their draws may start) one
-  // after another; within a row, positions from the last
-  const int b = order / upr, j = (upr - 1) - order % upr;
-  // kernel 2 may be scheduled once every CTA of this grid has started; it
-  // waits for each row's decision on its own
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int K = a.K, V = a.V;
   const bool verify = a.mode == kModeVerify;
   const long long u = static_cast<long long>(b) * (K + 1) + j;
@@ -1352,6 +1341,21 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) ssd_stats_kernel(const _
   }
 }
 
+// Kernel 1 of the two-kernel form (the draft side's ssd_saguaro_reweight):
+// one CTA per (unit, slice), rows in order so that rows are decided one
+// after another.
+template <typename TIn, bool kAligned, bool kGreedy>
+__global__ void __launch_bounds__(kThreads, kMinBlocks) ssd_stats_kernel(const __grid_constant__ Args a) {
+  const int S = a.n_slices;
+  const int order = blockIdx.x / S, slice = blockIdx.x % S;
+  const int upr = a.units_per_row;
+  const int b = order / upr, j = order % upr;
+  // kernel 2 may be scheduled once every CTA of this grid has started; it
+  // waits for each of its units' records on its own
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  stats_cta<TIn, kAligned, kGreedy>(a, b, j, slice);
+}
+
 // Shared memory of kernel 2.
 struct Smem2 {
   uint64_t full[kStages];
@@ -1402,15 +1406,16 @@ __device__ __forceinline__ void draw_vals(int draw, const TIn* baseP, long long 
   }
 }
 
+// One draw CTA: slice `slice` of draw unit du (verify: row du; reweight:
+// position du % K of row du / K).
 template <typename TIn, bool kAligned, bool kGreedy>
-__global__ void __launch_bounds__(kThreads, kMinBlocks) ssd_draw_kernel(const __grid_constant__ Args a) {
+__device__ __forceinline__ void draw_cta(const Args& a, int du, int slice) {
   constexpr int VE = Elem<TIn>::VE;
   extern __shared__ __align__(128) unsigned char ring_buf[];
   __shared__ __align__(16) Smem2 sm;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int S = a.d_slices;
-  const int du = blockIdx.x / S, slice = blockIdx.x % S;
   const int K = a.K, V = a.V;
   const bool verify = a.mode == kModeVerify;
 
@@ -1790,6 +1795,13 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) ssd_draw_kernel(const __
       a.c_next[static_cast<long long>(b) * K + i] = t;
     }
   }
+}
+
+// Kernel 2 of the two-kernel form: one CTA per (draw unit, slice).
+template <typename TIn, bool kAligned, bool kGreedy>
+__global__ void __launch_bounds__(kThreads, kMinBlocks) ssd_draw_kernel(const __grid_constant__ Args a) {
+  const int S = a.d_slices;
+  draw_cta<TIn, kAligned, kGreedy>(a, blockIdx.x / S, blockIdx.x % S);
 }
 
 }  // namespace ssd
