@@ -171,6 +171,25 @@ __device__ __forceinline__ void bulk_copy_g2s(void* dst, const void* src, uint32
       : "memory");
 }
 
+// The same copy with an L2 cache policy (see l2_policy_evict_first).
+__device__ __forceinline__ void bulk_copy_g2s_hint(void* dst, const void* src, uint32_t bytes, uint64_t* bar,
+                                                   uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], %4;" ::
+          "r"(smem_addr(dst)),
+      "l"(static_cast<uint64_t>(__cvta_generic_to_global(src))), "r"(bytes), "r"(smem_addr(bar)), "l"(policy)
+      : "memory");
+}
+
+// An L2 policy for data read once: its lines are the first to be evicted, so
+// a stream larger than L2 does not push out the small lines that are read
+// again soon (workspace records, flags).
+__device__ __forceinline__ uint64_t l2_policy_evict_first() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+
 // Split cluster barrier (all threads of every CTA of the cluster): arrive
 // with release semantics, wait with acquire semantics.  Every thread
 // alternates arrive and wait.
@@ -302,14 +321,22 @@ __device__ __forceinline__ float warp_max_nan(float v) {
 // high bit first.  `bits` = number of significant high bits of the keys.
 template <int kPerLane>
 __device__ __forceinline__ uint32_t warp_kth_largest(const uint32_t (&keys)[kPerLane], int F, int bits) {
+  // two bits per pass: the three extensions of the prefix are counted at once
+  // (bits is even), so the dependent chain is bits / 2 warp reductions long
   uint32_t prefix = 0u;
-  for (int bit = 31; bit >= 32 - bits; --bit) {
-    const uint32_t cand = prefix | (1u << bit);
-    int c = 0;
+  for (int bit = 30; bit >= 32 - bits; bit -= 2) {
+    const uint32_t c1 = prefix | (1u << bit), c2 = prefix | (2u << bit), c3 = prefix | (3u << bit);
+    int n1 = 0, n2 = 0, n3 = 0;
 #pragma unroll
-    for (int i = 0; i < kPerLane; ++i) c += keys[i] >= cand;
-    c = __reduce_add_sync(0xFFFFFFFFu, c);
-    if (c >= F) prefix = cand;
+    for (int i = 0; i < kPerLane; ++i) {
+      n1 += keys[i] >= c1;
+      n2 += keys[i] >= c2;
+      n3 += keys[i] >= c3;
+    }
+    n1 = __reduce_add_sync(0xFFFFFFFFu, n1);
+    n2 = __reduce_add_sync(0xFFFFFFFFu, n2);
+    n3 = __reduce_add_sync(0xFFFFFFFFu, n3);
+    prefix = n3 >= F ? c3 : (n2 >= F ? c2 : (n1 >= F ? c1 : prefix));
   }
   return prefix;
 }

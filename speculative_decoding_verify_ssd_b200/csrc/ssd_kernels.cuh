@@ -48,9 +48,10 @@ namespace ssd {
 
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
-constexpr int kMinBlocks = 4;          // CTAs per SM the register budget is set for
+constexpr int kMinBlocks = 5;          // statistics CTAs per SM the register budget is set for
+constexpr int kDrawMinBlocks = 4;      // draw CTAs per SM (their epilogue needs 64 registers)
 constexpr int kMaxSlices = 16;         // slices per logit row
-constexpr int kStages = 6;             // depth of the bulk-copy ring
+constexpr int kStages = 4;             // depth of the bulk-copy ring (32 KB: five CTAs per SM fit)
 constexpr int kChunkVecs = kThreads;   // 16-byte vectors per row per ring stage (draw kernel)
 constexpr int kStatsVPT = 2;           // stats kernel: vectors per thread per row per stage
 constexpr int kStatsChunkVecs = kChunkVecs * kStatsVPT;
@@ -76,6 +77,7 @@ constexpr int kFlagTimeout = SSD_ROW_DEVICE_TIMEOUT;
 constexpr size_t kRingBytes = static_cast<size_t>(kStages) * 2 * kChunkVecs * 16;
 
 static_assert(8 * (kCandCap + kGatherCap + kSelCap) <= kRingBytes, "merge buffers must fit in the idle ring");
+static_assert(2 * 4 * kMaxSlices * kMaxChunks * kWarps <= kRingBytes, "draw partial sums must fit in the idle ring");
 
 enum Mode : int { kModeVerify = 0, kModeReweight = 1 };
 enum Draw : int { kDrawNone = 0, kDrawResidual = 1, kDrawP = 2, kDrawQ = 3 };
@@ -254,6 +256,40 @@ __device__ __forceinline__ float consume_bf16(const uint4 w, int vbase, float c,
     s2 = f2_add(s2, f2_add(f2_add(e01, e23), f2_add(e45, e67)));
   }
   return vmax;
+}
+
+// Two vectors of one row from the same ring stage, softmax: both vector
+// maxima (returned for the top-F tracking), ONE rescale check for the pair,
+// then the packed exp2 sums.  A vector with ok = false is skipped (its words
+// read as -inf).
+__device__ __forceinline__ void consume2_bf16(const uint4 w0, const uint4 w1, bool ok0, bool ok1, float c, f32x2 c2,
+                                              float& m, f32x2& s2, f32x2& nm2, float& v0, float& v1) {
+  const uint32_t a = bf16x2_max_nan(bf16x2_max_nan(w0.x, w0.y), bf16x2_max_nan(w0.z, w0.w));
+  const uint32_t b = bf16x2_max_nan(bf16x2_max_nan(w1.x, w1.y), bf16x2_max_nan(w1.z, w1.w));
+  v0 = ok0 ? fmax_nan(bf16_lo(a), bf16_hi(a)) : -INFINITY;
+  v1 = ok1 ? fmax_nan(bf16_lo(b), bf16_hi(b)) : -INFINITY;
+  const float vmax = fmax_nan(v0, v1);
+  if (!(vmax <= m)) {  // a new maximum (or a NaN, which then sticks)
+    const float nm = fmax_nan(m, vmax);
+    const float sc = (m == -INFINITY) ? 0.f : ex2((m - nm) * c);  // s2 is 0 while m = -inf
+    s2 = f2_mul(s2, f2_pack(sc, sc));
+    m = nm;
+    const float nmc = -m * c;
+    nm2 = f2_pack(nmc, nmc);
+  }
+#pragma unroll
+  for (int v = 0; v < 2; ++v) {
+    if (v == 0 ? !ok0 : !ok1) continue;
+    const uint4 w = v == 0 ? w0 : w1;
+    float a0, a1, a2, a3, a4, a5, a6, a7;
+    f2_unpack(f2_fma(f2_pack(bf16_lo(w.x), bf16_hi(w.x)), c2, nm2), a0, a1);
+    f2_unpack(f2_fma(f2_pack(bf16_lo(w.y), bf16_hi(w.y)), c2, nm2), a2, a3);
+    f2_unpack(f2_fma(f2_pack(bf16_lo(w.z), bf16_hi(w.z)), c2, nm2), a4, a5);
+    f2_unpack(f2_fma(f2_pack(bf16_lo(w.w), bf16_hi(w.w)), c2, nm2), a6, a7);
+    const f32x2 e01 = f2_pack(ex2(a0), ex2(a1)), e23 = f2_pack(ex2(a2), ex2(a3));
+    const f32x2 e45 = f2_pack(ex2(a4), ex2(a5)), e67 = f2_pack(ex2(a6), ex2(a7));
+    s2 = f2_add(s2, f2_add(f2_add(e01, e23), f2_add(e45, e67)));
+  }
 }
 
 template <int VE, bool kGreedy>
@@ -522,7 +558,7 @@ __device__ __forceinline__ void fanout_row_power(float alpha_f, int K, int budge
 // and the warp that completes the count refills the stage with the chunk ST
 // ahead.  No CTA barrier sits in the stream, and no warp waits for the
 // slowest one except through the data it needs.
-template <typename TIn, int CV = kChunkVecs, int ST = kStages>
+template <typename TIn, int CV = kChunkVecs, int ST = kStages, bool kEvictFirst = false>
 struct Ring {
   unsigned char* buf;
   uint64_t* full;
@@ -540,8 +576,15 @@ struct Ring {
     const int v0 = c * CV;
     const int nv = min(CV, nvec - v0);
     mbar_arrive_expect_tx(&full[slot], static_cast<uint32_t>(nv) * 16u * static_cast<uint32_t>(nrows));
-    bulk_copy_g2s(stage(slot, 0), row0 + e0 + v0 * VE, static_cast<uint32_t>(nv) * 16u, &full[slot]);
-    if (nrows > 1) bulk_copy_g2s(stage(slot, 1), row1 + e0 + v0 * VE, static_cast<uint32_t>(nv) * 16u, &full[slot]);
+    if constexpr (kEvictFirst) {
+      const uint64_t pol = l2_policy_evict_first();
+      bulk_copy_g2s_hint(stage(slot, 0), row0 + e0 + v0 * VE, static_cast<uint32_t>(nv) * 16u, &full[slot], pol);
+      if (nrows > 1)
+        bulk_copy_g2s_hint(stage(slot, 1), row1 + e0 + v0 * VE, static_cast<uint32_t>(nv) * 16u, &full[slot], pol);
+    } else {
+      bulk_copy_g2s(stage(slot, 0), row0 + e0 + v0 * VE, static_cast<uint32_t>(nv) * 16u, &full[slot]);
+      if (nrows > 1) bulk_copy_g2s(stage(slot, 1), row1 + e0 + v0 * VE, static_cast<uint32_t>(nv) * 16u, &full[slot]);
+    }
     n_issued = c + 1;
   }
   __device__ __forceinline__ void start(int tid) {
@@ -754,7 +797,7 @@ __device__ __forceinline__ void stats_cta(const Args& a, int b, int j, int slice
   const int n = max(0, e1 - e0);
   const int nvec = (n + VE - 1) / VE;
   const int nch = (nvec + kStatsChunkVecs - 1) / kStatsChunkVecs;
-  Ring<TIn, kStatsChunkVecs, kStatsStages> ring;
+  Ring<TIn, kStatsChunkVecs, kStatsStages, true> ring;  // read once: first out of L2
   ring.buf = ring_buf;
   ring.full = sm.full;
   ring.rel = sm.rel;
@@ -833,51 +876,76 @@ __device__ __forceinline__ void stats_cta(const Args& a, int b, int j, int slice
   float vm1 = -INFINITY, vm2 = -INFINITY, vm3 = -INFINITY;  // top three vector maxima of the source row
   int g1 = -1, g2 = -1;
   uint4 keep1 = make_uint4(0u, 0u, 0u, 0u), keep2 = keep1;  // the source vectors holding vm1, vm2
-  for (int c = 0; c < nch; ++c) {
-    if constexpr (kAligned) ring.acquire(c, tid, tmo);
-#pragma unroll
-    for (int v = 0; v < kStatsVPT; ++v) {
-    const int t = v * kChunkVecs + tid;  // the thread's vector within the chunk
-    const int g = c * kStatsChunkVecs + t;
-    if (g < nvec) {
-      const int vbase = e0 + g * VE;
-      float vsrc;
-      uint4 wsrc = make_uint4(0u, 0u, 0u, 0u);
-      if constexpr (kAligned && sizeof(TIn) == 2) {
-        float vp = -INFINITY;
-        uint4 wq = make_uint4(0u, 0u, 0u, 0u), wp = wq;
-        if (hasP) { wp = ring.vec(c, slotP, t); vp = consume_bf16<kGreedy>(wp, vbase, cT, cT2, mP, sP2, nmP2, argP, nan_seen); }
-        float vq = -INFINITY;
-        if (hasQ) { wq = ring.vec(c, slotQ, t); vq = consume_bf16<kGreedy>(wq, vbase, cT, cT2, mQ, sQ2, nmQ2, argQ, nan_seen); }
-        vsrc = srcQ ? vq : vp;
-        wsrc = srcQ ? wq : wp;
+  auto track = [&](float vsrc, const uint4& wsrc, int g) {
+    if (vsrc > vm3) {
+      if (vsrc > vm2) {
+        vm3 = vm2;
+        if (vsrc > vm1) { vm2 = vm1; keep2 = keep1; g2 = g1; vm1 = vsrc; g1 = g; keep1 = wsrc; }
+        else { vm2 = vsrc; g2 = g; keep2 = wsrc; }
       } else {
-        float x[VE];
-        float vp = -INFINITY, vq = -INFINITY;
-        uint4 wp = make_uint4(0u, 0u, 0u, 0u), wq = wp;
-        if (hasP) {
-          if constexpr (kAligned) { wp = ring.vec(c, slotP, t); Elem<TIn>::unpack(wp, x); }
-          else load_group<TIn, false>(baseP, rbP, vbase, e1, x);
-          vp = consume_f<VE, kGreedy>(x, vbase, cT, mP, sP, nmP1, argP, nan_seen);
-        }
-        if (hasQ) {
-          if constexpr (kAligned) { wq = ring.vec(c, slotQ, t); Elem<TIn>::unpack(wq, x); }
-          else load_group<TIn, false>(baseQ, rbQ, vbase, e1, x);
-          vq = consume_f<VE, kGreedy>(x, vbase, cT, mQ, sQ, nmQ1, argQ, nan_seen);
-        }
-        vsrc = srcQ ? vq : vp;
-        wsrc = srcQ ? wq : wp;
-      }
-      if (vsrc > vm3) {
-        if (vsrc > vm2) {
-          vm3 = vm2;
-          if (vsrc > vm1) { vm2 = vm1; keep2 = keep1; g2 = g1; vm1 = vsrc; g1 = g; keep1 = wsrc; }
-          else { vm2 = vsrc; g2 = g; keep2 = wsrc; }
-        } else {
-          vm3 = vsrc;
-        }
+        vm3 = vsrc;
       }
     }
+  };
+  for (int c = 0; c < nch; ++c) {
+    if constexpr (kAligned) ring.acquire(c, tid, tmo);
+    if constexpr (kAligned && sizeof(TIn) == 2 && !kGreedy && kStatsVPT == 2) {
+      // both of the thread's vectors of each row in one go: one rescale check
+      // per row per stage
+      const int g0 = c * kStatsChunkVecs + tid, g1v = g0 + kChunkVecs;
+      const bool ok0 = g0 < nvec, ok1 = g1v < nvec;
+      const uint4 neg = make_uint4(0xFF80FF80u, 0xFF80FF80u, 0xFF80FF80u, 0xFF80FF80u);
+      uint4 wp0 = neg, wp1 = neg, wq0 = neg, wq1 = neg;
+      float vp0 = -INFINITY, vp1 = -INFINITY, vq0 = -INFINITY, vq1 = -INFINITY;
+      if (hasP) {
+        if (ok0) wp0 = ring.vec(c, slotP, tid);
+        if (ok1) wp1 = ring.vec(c, slotP, tid + kChunkVecs);
+        consume2_bf16(wp0, wp1, ok0, ok1, cT, cT2, mP, sP2, nmP2, vp0, vp1);
+      }
+      if (hasQ) {
+        if (ok0) wq0 = ring.vec(c, slotQ, tid);
+        if (ok1) wq1 = ring.vec(c, slotQ, tid + kChunkVecs);
+        consume2_bf16(wq0, wq1, ok0, ok1, cT, cT2, mQ, sQ2, nmQ2, vq0, vq1);
+      }
+      if (ok0) track(srcQ ? vq0 : vp0, srcQ ? wq0 : wp0, g0);
+      if (ok1) track(srcQ ? vq1 : vp1, srcQ ? wq1 : wp1, g1v);
+    } else {
+#pragma unroll
+      for (int v = 0; v < kStatsVPT; ++v) {
+        const int t = v * kChunkVecs + tid;  // the thread's vector within the chunk
+        const int g = c * kStatsChunkVecs + t;
+        if (g < nvec) {
+          const int vbase = e0 + g * VE;
+          float vsrc;
+          uint4 wsrc = make_uint4(0u, 0u, 0u, 0u);
+          if constexpr (kAligned && sizeof(TIn) == 2) {
+            float vp = -INFINITY;
+            uint4 wq = make_uint4(0u, 0u, 0u, 0u), wp = wq;
+            if (hasP) { wp = ring.vec(c, slotP, t); vp = consume_bf16<kGreedy>(wp, vbase, cT, cT2, mP, sP2, nmP2, argP, nan_seen); }
+            float vq = -INFINITY;
+            if (hasQ) { wq = ring.vec(c, slotQ, t); vq = consume_bf16<kGreedy>(wq, vbase, cT, cT2, mQ, sQ2, nmQ2, argQ, nan_seen); }
+            vsrc = srcQ ? vq : vp;
+            wsrc = srcQ ? wq : wp;
+          } else {
+            float x[VE];
+            float vp = -INFINITY, vq = -INFINITY;
+            uint4 wp = make_uint4(0u, 0u, 0u, 0u), wq = wp;
+            if (hasP) {
+              if constexpr (kAligned) { wp = ring.vec(c, slotP, t); Elem<TIn>::unpack(wp, x); }
+              else load_group<TIn, false>(baseP, rbP, vbase, e1, x);
+              vp = consume_f<VE, kGreedy>(x, vbase, cT, mP, sP, nmP1, argP, nan_seen);
+            }
+            if (hasQ) {
+              if constexpr (kAligned) { wq = ring.vec(c, slotQ, t); Elem<TIn>::unpack(wq, x); }
+              else load_group<TIn, false>(baseQ, rbQ, vbase, e1, x);
+              vq = consume_f<VE, kGreedy>(x, vbase, cT, mQ, sQ, nmQ1, argQ, nan_seen);
+            }
+            vsrc = srcQ ? vq : vp;
+            wsrc = srcQ ? wq : wp;
+          }
+          track(vsrc, wsrc, g);
+        }
+      }
     }
     if constexpr (kAligned) ring.release(c, lane);
   }
@@ -1433,15 +1501,16 @@ __device__ __forceinline__ void draw_cta(const Args& a, int du, int slice) {
   if (warp == 1 && (a.F != nullptr || a.alpha != nullptr)) load_plan(a, verify ? du : du / K, sm.s_F, lane);
   __syncthreads();
   const bool dep_ok = sm.dep_ok != 0;
-  // This CTA has read the epoch; the last CTA to do so advances it for the
-  // next call (off the path of threads 0..63, which start the stream).
-  if (tid == 2 * 32) {
-    if (atomicAdd(a.k2_done, 1) == static_cast<int>(gridDim.x) - 1) {
+  // Every CTA has read the epoch above; the last CTA of the grid to leave
+  // advances it for the next call.  Counted at each CTA's exit (thread 0), so
+  // the round trip never delays the stream.
+  auto leave = [&]() {
+    if (tid == 0 && atomicAdd(a.k2_done, 1) == static_cast<int>(gridDim.x) - 1) {
       *a.k2_done = 0;
       __threadfence();
       atomicAdd(a.epoch, 1u);
     }
-  }
+  };
 
   // ---- which unit this row (or draft position) draws from ----------------------------
   int b, j, rowflags = 0, draw;
@@ -1471,7 +1540,10 @@ __device__ __forceinline__ void draw_cta(const Args& a, int du, int slice) {
   const long long u = static_cast<long long>(b) * (K + 1) + j;
   const bool row_invalid = verify ? (rowflags & SSD_ROW_INVALID) != 0 : (st.flags & SSD_ROW_INVALID) != 0;
   const bool streams = !kGreedy && !row_invalid;
-  if (!streams && slice != 0) return;
+  if (!streams && slice != 0) {
+    leave();
+    return;
+  }
 
   const TIn *baseP, *baseQ;
   long long rbP, rbQ;
@@ -1561,7 +1633,10 @@ __device__ __forceinline__ void draw_cta(const Args& a, int du, int slice) {
     if constexpr (kAligned) ring.drain(tid, tmo);
     if (tid == 0) sm.is_last = arrive_acq_rel_gpu(a.draw_arrive + du) == S - 1;
     __syncthreads();
-    if (!sm.is_last) return;
+    if (!sm.is_last) {
+      leave();
+      return;
+    }
 
     // ============ the draw: the last slice of this unit to arrive ====================
     // Every slice's (chunk, warp) partial sums in one round trip, into the
@@ -1731,6 +1806,7 @@ __device__ __forceinline__ void draw_cta(const Args& a, int du, int slice) {
         a.row_arrive2[b] = 0;
       }
     }
+    leave();
     return;
   }
 
@@ -1795,11 +1871,12 @@ __device__ __forceinline__ void draw_cta(const Args& a, int du, int slice) {
       a.c_next[static_cast<long long>(b) * K + i] = t;
     }
   }
+  leave();
 }
 
 // Kernel 2 of the two-kernel form: one CTA per (draw unit, slice).
 template <typename TIn, bool kAligned, bool kGreedy>
-__global__ void __launch_bounds__(kThreads, kMinBlocks) ssd_draw_kernel(const __grid_constant__ Args a) {
+__global__ void __launch_bounds__(kThreads, kDrawMinBlocks) ssd_draw_kernel(const __grid_constant__ Args a) {
   const int S = a.d_slices;
   draw_cta<TIn, kAligned, kGreedy>(a, blockIdx.x / S, blockIdx.x % S);
 }
