@@ -182,6 +182,10 @@ static ssd_status make_plan(int V, int rows, int esize, long long units, Plan* p
   return SSD_OK;
 }
 
+static long long stats_grid(const Args& a) {
+  return static_cast<long long>(a.B) * a.units_per_row * a.n_slices;
+}
+
 static std::mutex g_attr_mu;
 static std::map<std::tuple<const void*, int>, int> g_attr_done;
 
@@ -201,8 +205,8 @@ static cudaError_t prepare_kernel(const void* fn) {
 // Workspace: slice partials, unit states, draw partials, row states, then the
 // counters (zero between calls) and the error word.
 struct WsLayout {
-  size_t parts, ustate, dparts, rstate, arrive1, row_arrive, draw_arrive, row_arrive2, rflag, epoch, k2_done, error,
-      total;
+  size_t parts, ustate, dparts, rstate, arrive1, row_arrive, draw_arrive, draw_owner, row_arrive2, rflag, uword, dtot,
+      epoch, k2_done, error, total;
   int n_slices;
 };
 
@@ -233,9 +237,12 @@ static WsLayout ws_layout(int B, int K, int V, int dtype) {
   w.dparts = off;      off = up256(off + nb * static_cast<size_t>(K) * ns * sizeof(DrawPart));
   w.rstate = off;      off = up256(off + nb * sizeof(RowState));
   w.rflag = off;       off += nb * static_cast<size_t>(K) * sizeof(uint64_t);  // 8-byte aligned here
+  w.uword = off;       off += units * sizeof(uint64_t);
+  w.dtot = off;        off += nb * static_cast<size_t>(K) * ns * sizeof(uint64_t);
   w.arrive1 = off;     off += units * sizeof(int32_t);
   w.row_arrive = off;  off += nb * sizeof(int32_t);
   w.draw_arrive = off; off += nb * static_cast<size_t>(K) * sizeof(int32_t);
+  w.draw_owner = off;  off += nb * static_cast<size_t>(K) * sizeof(int32_t);
   w.row_arrive2 = off; off += nb * sizeof(int32_t);
   w.epoch = off;       off += sizeof(uint32_t);
   w.k2_done = off;     off += sizeof(int32_t);
@@ -253,8 +260,11 @@ static void bind_workspace(Args& a, void* ws, const WsLayout& w) {
   a.arrive1 = reinterpret_cast<int32_t*>(base + w.arrive1);
   a.row_arrive = reinterpret_cast<int32_t*>(base + w.row_arrive);
   a.draw_arrive = reinterpret_cast<int32_t*>(base + w.draw_arrive);
+  a.draw_owner = reinterpret_cast<int32_t*>(base + w.draw_owner);
   a.row_arrive2 = reinterpret_cast<int32_t*>(base + w.row_arrive2);
   a.rflag = reinterpret_cast<uint64_t*>(base + w.rflag);
+  a.uword = reinterpret_cast<uint64_t*>(base + w.uword);
+  a.dtot = reinterpret_cast<uint64_t*>(base + w.dtot);
   a.epoch = reinterpret_cast<uint32_t*>(base + w.epoch);
   a.k2_done = reinterpret_cast<int32_t*>(base + w.k2_done);
   a.error = reinterpret_cast<int32_t*>(base + w.error);
@@ -267,7 +277,7 @@ static ssd_status launch_t(const Args& a, long long units, long long draw_units,
   if (prepare_kernel(f1) != cudaSuccess || prepare_kernel(f2) != cudaSuccess) return SSD_ERR_CUDA;
   const size_t smem = kRingBytes;  // the ring, and afterwards the merge buffers
   ssd_stats_kernel<TIn, kAligned, kGreedy>
-      <<<static_cast<unsigned>(units * a.n_slices), kThreads, smem, stream>>>(a);
+      <<<static_cast<unsigned>(stats_grid(a)), kThreads, smem, stream>>>(a);
   if (cudaGetLastError() != cudaSuccess) return SSD_ERR_CUDA;
   if (draw_units > 0) {
     // Programmatic dependent launch: the draw kernel may start while the
@@ -408,7 +418,6 @@ ssd_status ssd_verify(const void* target_logits, const void* draft_logits, const
   const ssd_status ps = make_plan(V, 2, esize, units, &plan);
   if (ps != SSD_OK) return ps;
   if (plan.n_slices > wl.n_slices) return SSD_ERR_WORKSPACE;
-  if (units * plan.n_slices > 0x7FFFFFFFLL) return SSD_ERR_INVALID_ARG;
   Args a = {};
   a.target = target_logits;
   a.draft = draft_logits;
@@ -419,7 +428,9 @@ ssd_status ssd_verify(const void* target_logits, const void* draft_logits, const
   a.alpha = F ? nullptr : alpha;
   a.fanout_mode = fanout_mode;
   a.B = B; a.K = K; a.V = V; a.budget = budget; a.mode = kModeVerify;
-  a.n_slices = plan.n_slices; a.chunk = plan.chunk; a.units_per_row = K + 1; a.draws = 1;
+  a.units_per_row = K + 1; a.draws = 1;
+  a.n_slices = plan.n_slices; a.chunk = plan.chunk;
+  if (stats_grid(a) > 0x7FFFFFFFLL) return SSD_ERR_INVALID_ARG;
   Plan dplan;
   const ssd_status dps = make_plan(V, 2, esize, B, &dplan, kDrawCtaBytes);
   if (dps != SSD_OK) return dps;

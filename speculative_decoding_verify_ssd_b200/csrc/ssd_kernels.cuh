@@ -48,12 +48,21 @@ namespace ssd {
 
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
-constexpr int kMinBlocks = 5;          // statistics CTAs per SM the register budget is set for
+#ifndef SSD_MIN_BLOCKS
+#define SSD_MIN_BLOCKS 5
+#endif
+#ifndef SSD_STAGES
+#define SSD_STAGES 4
+#endif
+#ifndef SSD_STATS_VPT
+#define SSD_STATS_VPT 2
+#endif
+constexpr int kMinBlocks = SSD_MIN_BLOCKS;  // statistics CTAs per SM the register budget is set for
 constexpr int kDrawMinBlocks = 4;      // draw CTAs per SM (their epilogue needs 64 registers)
 constexpr int kMaxSlices = 16;         // slices per logit row
-constexpr int kStages = 4;             // depth of the bulk-copy ring (32 KB: five CTAs per SM fit)
+constexpr int kStages = SSD_STAGES;    // depth of the bulk-copy ring (32 KB: five CTAs per SM fit)
 constexpr int kChunkVecs = kThreads;   // 16-byte vectors per row per ring stage (draw kernel)
-constexpr int kStatsVPT = 2;           // stats kernel: vectors per thread per row per stage
+constexpr int kStatsVPT = SSD_STATS_VPT;  // stats kernel: vectors per thread per row per stage
 constexpr int kStatsChunkVecs = kChunkVecs * kStatsVPT;
 constexpr int kStatsStages = kStages * kChunkVecs / kStatsChunkVecs;  // same ring bytes
 constexpr int kMaxChunks = 16;         // ring chunks per slice
@@ -166,9 +175,12 @@ struct Args {
   RowState* rstate;
   int32_t* arrive1;
   int32_t* row_arrive;
-  int32_t* draw_arrive;
+  int32_t* draw_arrive;    // per draw unit: slices that published their masses
+  int32_t* draw_owner;     // per draw unit: the tag of the last call whose row a CTA took to finish
+  uint64_t* dtot;          // per (draw unit, slice): (epoch + 1) << 32 | bits of the slice's mass
   int32_t* row_arrive2;
-  uint64_t* rflag;         // per draw unit, once the row decision is written: (epoch + 1) << 32 | k* << 8 | flags
+  uint64_t* rflag;         // reweight, per draft position: (epoch + 1) << 32 | flags, once the row is decided
+  uint64_t* uword;         // verify, per unit: (epoch + 1) << 32 | near << 17 | rejected << 16 | pflags << 8 | flags
   uint32_t* epoch;         // calls completed on this workspace (kernel 2 advances it)
   int32_t* k2_done;        // kernel 2 CTAs past their wait
   int32_t* error;
@@ -772,13 +784,12 @@ struct Smem1 {
 
 // One statistics CTA: slice `slice` of unit (row b, position j).
 template <typename TIn, bool kAligned, bool kGreedy>
-__device__ __forceinline__ void stats_cta(const Args& a, int b, int j, int slice) {
+__device__ __forceinline__ void stats_cta(const Args& a, int b, int j, int slice, int S, int chunk) {
   constexpr int VE = Elem<TIn>::VE;
   extern __shared__ __align__(128) unsigned char ring_buf[];
   __shared__ __align__(16) Smem1 sm;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int S = a.n_slices;
   const int upr = a.units_per_row;
   const int K = a.K, V = a.V;
   const bool verify = a.mode == kModeVerify;
@@ -792,8 +803,8 @@ __device__ __forceinline__ void stats_cta(const Args& a, int b, int j, int slice
   const bool has_d = verify && j < K;
 
   // ---- slice [e0, e1) of the rows, vectors of VE elements --------------------------
-  const int e0 = slice * a.chunk;
-  const int e1 = min(V, e0 + a.chunk);
+  const int e0 = slice * chunk;
+  const int e1 = min(V, e0 + chunk);
   const int n = max(0, e1 - e0);
   const int nvec = (n + VE - 1) / VE;
   const int nch = (nvec + kStatsChunkVecs - 1) / kStatsChunkVecs;
@@ -1015,7 +1026,7 @@ __device__ __forceinline__ void stats_cta(const Args& a, int b, int j, int slice
   if (plan_bad) flags |= SSD_ROW_BAD_PLAN;
   const bool want_topf = has_plan && Fj > 0;
   const bool fast_ok = want_topf && Fj <= kMaxGroups;
-  SlicePart* part = a.parts + u * S + slice;
+  SlicePart* part = a.parts + u * a.n_slices + slice;
   if (warp == 0) {
     float m1 = -INFINITY, s1 = 0.f, m2 = -INFINITY, s2 = 0.f;
     int a1 = INT_MAX, a2 = INT_MAX;
@@ -1139,7 +1150,7 @@ __device__ __forceinline__ void stats_cta(const Args& a, int b, int j, int slice
 #endif
 
   // =============== the unit's finalizer: its last slice, once all have arrived ======
-  const SlicePart* parts = a.parts + u * S;
+  const SlicePart* parts = a.parts + u * a.n_slices;
   // Every slice's published candidates, loaded at once with the statistics
   // (slot c * cap + r holds candidate r of slice c; entries past a slice's
   // count are ignored).
@@ -1167,7 +1178,7 @@ __device__ __forceinline__ void stats_cta(const Args& a, int b, int j, int slice
       xp = __ldcg(&parts[lane].xdP);
       xq = __ldcg(&parts[lane].xdQ);
     }
-    const int cd = (has_d && d >= 0 && d < V) ? d / a.chunk : 0;  // the slice holding d
+    const int cd = (has_d && d >= 0 && d < V) ? d / chunk : 0;  // the slice holding d
     xp = __shfl_sync(0xFFFFFFFFu, xp, cd);
     xq = __shfl_sync(0xFFFFFFFFu, xq, cd);
     const int cnt = min(min(nc, Fj), kCandSlice);
@@ -1206,9 +1217,11 @@ __device__ __forceinline__ void stats_cta(const Args& a, int b, int j, int slice
   __syncthreads();
   const float MP = sm.MP, MQ = sm.MQ, SP = sm.SP, SQ = sm.SQ;
   if (sm.tmo || !arrivals_ok) flags |= kFlagTimeout;
-  if (hasP && !(MP > -INFINITY && MP < INFINITY)) flags |= SSD_ROW_NONFINITE;
+  // a non-finite target row is kept apart (pflags): the row decision may
+  // count it only for the positions the outcome depends on
+  const int pflags = (hasP && !(MP > -INFINITY && MP < INFINITY)) ? SSD_ROW_NONFINITE : 0;
   if (hasQ && !(MQ > -INFINITY && MQ < INFINITY)) flags |= SSD_ROW_NONFINITE;
-  const bool valid = (flags & SSD_ROW_INVALID) == 0;
+  const bool valid = ((flags | pflags) & SSD_ROW_INVALID) == 0;
   const bool slow = want_topf && valid && (!one_round || sm.slow != 0);
   Cand* sel = gbuf + kGatherCap;
   const float nmP = -MP * cT, nmQ = -MQ * cT;
@@ -1308,12 +1321,25 @@ __device__ __forceinline__ void stats_cta(const Args& a, int b, int j, int slice
     UnitState st;
     st.MP = MP; st.SP = SP; st.MQ = MQ; st.SQ = SQ;
     st.Z = Z; st.bx = bx; st.a = acc; st.amargin = amargin;
-    st.bi = bi; st.argP = sm.argP; st.argQ = sm.argQ; st.flags = flags;
+    st.bi = bi; st.argP = sm.argP; st.argQ = sm.argQ; st.flags = flags | pflags;
     st.rejected = rejected; st.Fj = Fj; st.seg_off = seg_off; st.dmargin = INFINITY;
     a.ustate[u] = st;
     a.arrive1[u] = 0;
   }
   __syncthreads();
+  if (verify) {
+    // The unit's result in one tagged word: the draw CTAs of the row read the
+    // row's K+1 words and take the decision themselves (k* = the first
+    // rejected position), so no CTA here waits for the rest of the row.
+    if (tid == 0) {
+      const uint64_t tag = *reinterpret_cast<volatile uint32_t*>(a.epoch) + 1u;
+      const uint32_t lo = static_cast<uint32_t>(flags & 0xFF) | static_cast<uint32_t>(pflags & 0xFF) << 8 |
+                          static_cast<uint32_t>(rejected ? 1 : 0) << 16 |
+                          static_cast<uint32_t>(amargin < kNearTie ? 1 : 0) << 17;
+      st_release_gpu_u64(a.uword + u, tag << 32 | lo);
+    }
+    return;
+  }
 #if SSD_LAST_ARRIVES
   // Likewise per row: the last unit of the row to arrive decides.
   if (tid == 0) sm.is_last_row = arrive_acq_rel_gpu(a.row_arrive + b) == upr - 1 ? 1 : 0;
@@ -1421,7 +1447,7 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) ssd_stats_kernel(const _
   // kernel 2 may be scheduled once every CTA of this grid has started; it
   // waits for each of its units' records on its own
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-  stats_cta<TIn, kAligned, kGreedy>(a, b, j, slice);
+  stats_cta<TIn, kAligned, kGreedy>(a, b, j, slice, S, a.chunk);
 }
 
 // Shared memory of kernel 2.
@@ -1432,9 +1458,65 @@ struct Smem2 {
   float rs[kMaxChunks][kWarps];
   float ps[kMaxChunks][kWarps];
   int32_t s_F[SSD_MAX_K + 1];
-  float tl, total, margin;
-  int32_t cstar, use_p, drawn, is_last, is_last_row, slot, tmo;
+  float tl, total, margin, myR;
+  int32_t cstar, use_p, drawn, is_last, is_last_row, slot, tmo, all_in, own;
 };
+
+// The draw's mass at the 8 tokens of one bf16 vector (of p and/or q), token
+// v0 first.  The arithmetic of each token is draw_vals' scalar form, two
+// tokens per packed instruction; the Saguaro set test runs only for a vector
+// whose largest draft logit reaches the set's boundary logit bx.
+__device__ __forceinline__ void draw_vals_bf16(int draw, uint4 wp, uint4 wq, int v0, float cT, float nmP, float nmQ,
+                                               float invSP, float wS, float wN, bool check_S, float bx, int bi,
+                                               bool use_p, float (&val)[8], float (&pv)[8]) {
+  const f32x2 c2 = f2_pack(cT, cT);
+  const uint32_t wpw[4] = {wp.x, wp.y, wp.z, wp.w};
+  const uint32_t wqw[4] = {wq.x, wq.y, wq.z, wq.w};
+  float pp[8], qq[8];
+  if (draw != kDrawQ) {
+    const f32x2 n2 = f2_pack(nmP, nmP), s2 = f2_pack(invSP, invSP);
+#pragma unroll
+    for (int h = 0; h < 4; ++h) {
+      float a0, a1;
+      f2_unpack(f2_fma(f2_pack(bf16_lo(wpw[h]), bf16_hi(wpw[h])), c2, n2), a0, a1);
+      f2_unpack(f2_mul(f2_pack(ex2(a0), ex2(a1)), s2), pp[2 * h], pp[2 * h + 1]);
+    }
+  }
+  if (draw != kDrawP) {
+    bool anyS = false;
+    if (check_S) {
+      const uint32_t m2 = bf16x2_max_nan(bf16x2_max_nan(wq.x, wq.y), bf16x2_max_nan(wq.z, wq.w));
+      anyS = fmax_nan(bf16_lo(m2), bf16_hi(m2)) >= bx;
+    }
+    const f32x2 n2 = f2_pack(nmQ, nmQ);
+#pragma unroll
+    for (int h = 0; h < 4; ++h) {
+      const float x0 = bf16_lo(wqw[h]), x1 = bf16_hi(wqw[h]);
+      float w0 = wN, w1 = wN;
+      if (anyS) {
+        const int v = v0 + 2 * h;
+        if (x0 > bx || (x0 == bx && v <= bi)) w0 = wS;
+        if (x1 > bx || (x1 == bx && v + 1 <= bi)) w1 = wS;
+      }
+      float a0, a1;
+      f2_unpack(f2_fma(f2_pack(x0, x1), c2, n2), a0, a1);
+      f2_unpack(f2_mul(f2_pack(ex2(a0), ex2(a1)), f2_pack(w0, w1)), qq[2 * h], qq[2 * h + 1]);
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    if (draw == kDrawResidual) {
+      val[i] = use_p ? pp[i] : fmaxf(pp[i] - qq[i], 0.f);
+      pv[i] = pp[i];
+    } else if (draw == kDrawP) {
+      val[i] = pp[i];
+      pv[i] = 0.f;
+    } else {
+      val[i] = qq[i];
+      pv[i] = 0.f;
+    }
+  }
+}
 
 // The draw's mass at VE consecutive tokens of vector g of slice [e0, e1).
 template <typename TIn, bool kAligned>
@@ -1444,6 +1526,13 @@ __device__ __forceinline__ void draw_vals(int draw, const TIn* baseP, long long 
                                           float bx, int bi, bool use_p, float (&val)[Elem<TIn>::VE],
                                           float (&pv)[Elem<TIn>::VE]) {
   constexpr int VE = Elem<TIn>::VE;
+  if constexpr (kAligned && sizeof(TIn) == 2) {
+    uint4 wp = make_uint4(0u, 0u, 0u, 0u), wq = wp;
+    if (draw != kDrawQ) wp = wp_ring ? *wp_ring : ld_vec(baseP + rbP + e0 + g * VE);
+    if (draw != kDrawP) wq = wq_ring ? *wq_ring : ld_vec(baseQ + rbQ + e0 + g * VE);
+    draw_vals_bf16(draw, wp, wq, e0 + g * VE, cT, nmP, nmQ, invSP, wS, wN, check_S, bx, bi, use_p, val, pv);
+    return;
+  }
   float xp[VE], xq[VE];
   if (draw != kDrawQ) {
     if (wp_ring) Elem<TIn>::unpack(*wp_ring, xp);
@@ -1488,12 +1577,41 @@ __device__ __forceinline__ void draw_cta(const Args& a, int du, int slice) {
   const bool verify = a.mode == kModeVerify;
 
   // ---- the row decision this CTA needs (kernel 1 may still be running) -------------
-  if (tid == 0) {
+  if (verify) {
+    // Lane k waits for unit k's tagged word (lane 0 also for unit 32 when
+    // K = 32); k* is the first rejected position, else K.
+    if (warp == 0) {
+      const uint32_t epoch = *reinterpret_cast<volatile const uint32_t*>(a.epoch);
+      const int upr = K + 1;
+      const uint64_t* uw = a.uword + static_cast<long long>(du) * upr;
+      uint64_t w0 = 0, w1 = 0;
+      bool ok = true;
+      if (lane < upr) ok = wait_tagged(uw + lane, epoch + 1u, kDepWaitNs, &w0);
+      if (lane + 32 < upr) ok = wait_tagged(uw + lane + 32, epoch + 1u, kDepWaitNs, &w1) && ok;
+      const bool all_ok = __all_sync(0xFFFFFFFFu, ok);
+      const uint32_t lo0 = static_cast<uint32_t>(w0), lo1 = static_cast<uint32_t>(w1);
+      const unsigned rm = __ballot_sync(0xFFFFFFFFu, lane < K && ((lo0 >> 16) & 1u));
+      const int kstar = rm ? __ffs(rm) - 1 : K;
+      // flags of every unit; a non-finite target row, a near-tie accept test
+      // only up to k*
+      uint32_t f = (lo0 | lo1) & 0xFFu;
+      f |= (lo0 >> 8) & 0xFFu;
+      f |= (lo1 >> 8) & 0xFFu;
+      if (lane <= kstar && ((lo0 >> 17) & 1u)) f |= SSD_ROW_NEAR_TIE;
+      f = __reduce_or_sync(0xFFFFFFFFu, f);
+      if (lane == 0) {
+        sm.dep_ok = all_ok ? 1 : 0;
+        if (!all_ok) atomicExch(a.error, 1);
+        sm.w_kstar = kstar;
+        sm.w_flags = static_cast<int32_t>(f);
+      }
+    }
+  } else if (tid == 0) {
     const uint32_t epoch = *reinterpret_cast<volatile const uint32_t*>(a.epoch);
     uint64_t word = 0;
     sm.dep_ok = wait_tagged(a.rflag + du, epoch + 1u, kDepWaitNs, &word) ? 1 : 0;
     if (!sm.dep_ok) atomicExch(a.error, 1);
-    sm.w_kstar = static_cast<int32_t>((word >> 8) & 0xFF);  // the decision itself travels with the flag
+    sm.w_kstar = static_cast<int32_t>((word >> 8) & 0xFF);
     sm.w_flags = static_cast<int32_t>(word & 0xFF);
   }
   // The row's fan-out plan depends on the inputs only: form it while the
@@ -1568,12 +1686,11 @@ __device__ __forceinline__ void draw_cta(const Args& a, int du, int slice) {
   const int slotP = 0, slotQ = useP ? 1 : 0;
   if (kAligned && streams) ring.start(tid);
   if (verify) {  // the statistics of unit k*, while the first chunks are in flight
-    const RowState* rs = a.rstate + b;
-    amargin = __ldcg(&rs->amargin);
-    st.MP = __ldcg(&rs->MP); st.SP = __ldcg(&rs->SP); st.MQ = __ldcg(&rs->MQ); st.SQ = __ldcg(&rs->SQ);
-    st.Z = __ldcg(&rs->Z); st.bx = __ldcg(&rs->bx); st.bi = __ldcg(&rs->bi); st.argP = __ldcg(&rs->argP);
+    const UnitState* us = a.ustate + static_cast<long long>(b) * (K + 1) + j;
+    st.MP = __ldcg(&us->MP); st.SP = __ldcg(&us->SP); st.MQ = __ldcg(&us->MQ); st.SQ = __ldcg(&us->SQ);
+    st.Z = __ldcg(&us->Z); st.bx = __ldcg(&us->bx); st.bi = __ldcg(&us->bi); st.argP = __ldcg(&us->argP);
     st.argQ = 0;
-    st.Fj = __ldcg(&rs->Fj);
+    st.Fj = __ldcg(&us->Fj);
     st.flags = rowflags;
   }
 
@@ -1614,6 +1731,9 @@ __device__ __forceinline__ void draw_cta(const Args& a, int du, int slice) {
       if constexpr (kAligned) ring.release(c, lane);
     }
     tmo = __syncthreads_or(tmo);
+    // A slice that never wrapped the ring is still whole in shared memory:
+    // its CTA finds the row's crossing there, with no second read.
+    const bool resident = kAligned && nch <= kStages;
     if (warp == 0) {  // the slice's masses: lane l sums entries l, l + 32, ... then a butterfly
       float R = 0.f, RP = 0.f;
       for (int i = lane; i < nch * kWarps; i += 32) { R += sm.rs[i / kWarps][i % kWarps]; RP += sm.ps[i / kWarps][i % kWarps]; }
@@ -1623,32 +1743,17 @@ __device__ __forceinline__ void draw_cta(const Args& a, int du, int slice) {
         dparts[slice].R = R;
         dparts[slice].RP = RP;
         dparts[slice].timeout = tmo;
+        sm.myR = tmo ? __int_as_float(0x7FC00000) : R;
       }
     }
-    for (int i = tid; i < nch * kWarps; i += kThreads) {
-      dparts[slice].rs[i / kWarps][i % kWarps] = sm.rs[i / kWarps][i % kWarps];
-      dparts[slice].ps[i / kWarps][i % kWarps] = sm.ps[i / kWarps][i % kWarps];
+    if (!resident) {
+      for (int i = tid; i < nch * kWarps; i += kThreads) {
+        dparts[slice].rs[i / kWarps][i % kWarps] = sm.rs[i / kWarps][i % kWarps];
+        dparts[slice].ps[i / kWarps][i % kWarps] = sm.ps[i / kWarps][i % kWarps];
+      }
     }
-    __syncthreads();
-    if constexpr (kAligned) ring.drain(tid, tmo);
-    if (tid == 0) sm.is_last = arrive_acq_rel_gpu(a.draw_arrive + du) == S - 1;
-    __syncthreads();
-    if (!sm.is_last) {
-      leave();
-      return;
-    }
-
-    // ============ the draw: the last slice of this unit to arrive ====================
-    // Every slice's (chunk, warp) partial sums in one round trip, into the
-    // idle ring; the row's cache segment k* alongside.
-    const int nchm = ((a.d_chunk + VE - 1) / VE + kChunkVecs - 1) / kChunkVecs;  // chunks of a full slice
-    float* const Lrs = reinterpret_cast<float*>(ring_buf);
-    float* const Lps = Lrs + S * nchm * kWarps;
-    for (int i = tid; i < S * nchm * kWarps; i += kThreads) {
-      const int s2 = i / (nchm * kWarps), cw = i - s2 * (nchm * kWarps);
-      Lrs[i] = __ldcg(&dparts[s2].rs[cw / kWarps][cw % kWarps]);  // past a short slice's chunks: never read
-      Lps[i] = __ldcg(&dparts[s2].ps[cw / kWarps][cw % kWarps]);
-    }
+    // the row's cache segment k*, for the lookup (prefetched by every CTA
+    // that may finish the row)
     if (verify && a.c_tokens && !row_invalid) {
       int off = 0;
       for (int k = 0; k < j; ++k) off += sm.s_F[k];
@@ -1657,7 +1762,12 @@ __device__ __forceinline__ void draw_cta(const Args& a, int du, int slice) {
       if (tid < Fk) seg_tok0 = __ldcg(seg + tid);
       if (tid + kThreads < Fk) seg_tok1 = __ldcg(seg + tid + kThreads);
     }
-    if (warp == 0) {
+    __syncthreads();
+    if constexpr (kAligned) ring.drain(tid, tmo);
+
+    // Warp 0: the row's total and the slice where the cumulative mass crosses
+    // u * total (the first with prefix + part > t, else the last with mass).
+    auto find_slice = [&]() {
       float rp = 0.f, pp = 0.f;
       int to = 0;
       if (lane < S) {
@@ -1673,7 +1783,6 @@ __device__ __forceinline__ void draw_cta(const Args& a, int du, int slice) {
       const int use_p = (draw == kDrawResidual && !(R > 0.f)) ? 1 : 0;
       const float total = use_p ? RP : R;
       const float t = u_draw * total;
-      // crossing slice: the first with prefix + part > t, else the last with mass
       float run = 0.f, pre = 0.f, prelast = 0.f;
       int cstar = -1, clast = 0;
       for (int c = 0; c < S; ++c) {
@@ -1691,12 +1800,13 @@ __device__ __forceinline__ void draw_cta(const Args& a, int du, int slice) {
         sm.use_p = use_p;
         sm.tmo = anyto ? 1 : 0;
       }
-    }
-    __syncthreads();
-    if (warp == 0) {
+    };
+    // Warp 0, within slice s_star: chunk, warp, lane and token of the
+    // crossing, from that slice's (chunk, warp) sums Ls; the lane level reads
+    // the crossing warp-chunk from the ring (resident) or again from memory.
+    auto scan_slice = [&](const float* Ls, bool from_ring) {
       const int s_star = sm.cstar;
       const bool use_p = sm.use_p != 0;
-      const float* Ls = (use_p ? Lps : Lrs) + s_star * nchm * kWarps;
       const int e0s = s_star * a.d_chunk;
       const int e1s = min(V, e0s + a.d_chunk);
       const int nvs = (max(0, e1s - e0s) + VE - 1) / VE;
@@ -1731,12 +1841,18 @@ __device__ __forceinline__ void draw_cta(const Args& a, int du, int slice) {
       }
       if (w_star < 0) { w_star = w_last; pre_w = pre_last; }
       const float tl3 = tl2 - pre_w;
-      // lane level: the 32 vectors of that warp in that chunk, re-read from L2
+      // lane level: the 32 vectors of that warp in that chunk
       const int g = k_star * kChunkVecs + w_star * 32 + lane;
       float val[VE], pv[VE];
       if (g < nvs) {
-        draw_vals<TIn, kAligned>(draw, baseP, rbP, baseQ, rbQ, e0s, e1s, g, nullptr, nullptr, cT, nmP, nmQ, invSP, wS,
-                                 wN, check_S, st.bx, st.bi, use_p, val, pv);
+        const uint4* rp = nullptr;
+        const uint4* rq = nullptr;
+        if (from_ring) {
+          if (useP) rp = reinterpret_cast<const uint4*>(ring.stage(k_star % kStages, slotP) + (w_star * 32 + lane) * 16);
+          if (useQ) rq = reinterpret_cast<const uint4*>(ring.stage(k_star % kStages, slotQ) + (w_star * 32 + lane) * 16);
+        }
+        draw_vals<TIn, kAligned>(draw, baseP, rbP, baseQ, rbQ, e0s, e1s, g, rp, rq, cT, nmP, nmQ, invSP, wS, wN,
+                                 check_S, st.bx, st.bi, use_p, val, pv);
       } else {
 #pragma unroll
         for (int i = 0; i < VE; ++i) val[i] = 0.f;
@@ -1769,9 +1885,106 @@ __device__ __forceinline__ void draw_cta(const Args& a, int du, int slice) {
         sm.drawn = min(max(v, 0), V - 1);
         sm.margin = fminf(fabsf(lo), fabsf(hi)) / sm.total;
       }
+    };
+
+    if (resident) {
+      // Each slice publishes its mass in one tagged word, (epoch + 1) << 32 |
+      // bits(R) (NaN when its copies timed out); every slice of the row polls
+      // all S words (bounded), so all find the same crossing slice at once,
+      // and its CTA, which still holds the slice, finishes the row.  A CTA
+      // whose poll gives up may finish the row instead, as a timed-out row;
+      // an atomic maximum with the call's tag on the row's owner word lets
+      // exactly one CTA write the row.
+      const uint32_t tag = *reinterpret_cast<volatile const uint32_t*>(a.epoch) + 1u;
+      uint64_t* const dtot = a.dtot + static_cast<long long>(du) * S;
+      if (warp == 0) {
+        if (lane == 0) {
+          st_release_gpu_u64(dtot + slice, static_cast<uint64_t>(tag) << 32 | __float_as_uint(sm.myR));
+        }
+        uint64_t wv = 0;
+        bool ok = true;
+        if (lane < S) ok = wait_tagged(dtot + lane, tag, kDepWaitNs, &wv);
+        const bool all_ok = __all_sync(0xFFFFFFFFu, ok);
+        if (all_ok) {
+          const float rp = lane < S ? __uint_as_float(static_cast<uint32_t>(wv)) : 0.f;
+          float R = 0.f;
+          for (int c = 0; c < S; ++c) R += __shfl_sync(0xFFFFFFFFu, rp, c);
+          const int use_p = (draw == kDrawResidual && !(R > 0.f) && R == R) ? 1 : 0;
+          float pp = 0.f;
+          if (use_p && lane < S) pp = __ldcg(&dparts[lane].RP);  // rare: the row's residual is 0
+          float RP = 0.f;
+          for (int c = 0; c < S; ++c) RP += __shfl_sync(0xFFFFFFFFu, pp, c);
+          const float total = use_p ? RP : R;
+          const float t = u_draw * total;
+          float run = 0.f, pre = 0.f, prelast = 0.f;
+          int cstar = -1, clast = 0;
+          for (int c = 0; c < S; ++c) {
+            const float part = __shfl_sync(0xFFFFFFFFu, use_p ? pp : rp, c);
+            if (part > 0.f) { clast = c; prelast = run; }
+            if (cstar < 0 && run + part > t) { cstar = c; pre = run; }
+            run += part;
+          }
+          if (cstar < 0) { cstar = clast; pre = prelast; }
+          if (lane == 0) {
+            sm.cstar = cstar;
+            sm.tl = t - pre;
+            sm.total = total;
+            sm.use_p = use_p;
+            sm.tmo = (R == R) ? 0 : 1;  // a slice's copies timed out
+            sm.all_in = 1;
+          }
+        } else if (lane == 0) {
+          atomicExch(a.error, 1);
+          sm.cstar = -1;
+          sm.tmo = 1;
+          sm.total = 1.f;
+          sm.use_p = 0;
+          sm.all_in = 0;
+        }
+      }
+      __syncthreads();
+      const bool all_in = sm.all_in != 0;
+      const bool cand = !all_in || sm.tmo != 0 || sm.cstar == slice;
+      if (cand && tid == 0)
+        sm.own = atomicMax(reinterpret_cast<unsigned int*>(a.draw_owner) + du, tag) < tag ? 1 : 0;
+      __syncthreads();
+      const bool own = cand && sm.own != 0;
+      if (!own) {
+        leave();
+        return;
+      }
+      if (all_in && sm.tmo == 0) {
+        if (warp == 0) scan_slice(sm.use_p ? &sm.ps[0][0] : &sm.rs[0][0], true);
+      } else if (tid == 0) {
+        sm.drawn = -1;
+        sm.margin = INFINITY;
+        sm.tmo = 1;
+      }
+      __syncthreads();
+    } else {
+      if (tid == 0) sm.is_last = arrive_acq_rel_gpu(a.draw_arrive + du) == S - 1;
+      __syncthreads();
+      if (!sm.is_last) {
+        leave();
+        return;
+      }
+      // ============ the draw: the last slice of this unit to arrive ==================
+      // Every slice's (chunk, warp) partial sums in one round trip, into the
+      // idle ring.
+      const int nchm = ((a.d_chunk + VE - 1) / VE + kChunkVecs - 1) / kChunkVecs;  // chunks of a full slice
+      float* const Lrs = reinterpret_cast<float*>(ring_buf);
+      float* const Lps = Lrs + S * nchm * kWarps;
+      for (int i = tid; i < S * nchm * kWarps; i += kThreads) {
+        const int s2 = i / (nchm * kWarps), cw = i - s2 * (nchm * kWarps);
+        Lrs[i] = __ldcg(&dparts[s2].rs[cw / kWarps][cw % kWarps]);  // past a short slice's chunks: never read
+        Lps[i] = __ldcg(&dparts[s2].ps[cw / kWarps][cw % kWarps]);
+      }
+      if (warp == 0) find_slice();
+      __syncthreads();
+      if (warp == 0) scan_slice((sm.use_p ? Lps : Lrs) + sm.cstar * nchm * kWarps, false);
+      __syncthreads();
+      if (tid == 0) a.draw_arrive[du] = 0;
     }
-    __syncthreads();
-    if (tid == 0) a.draw_arrive[du] = 0;
   } else {
     // No stream: greedy (the argmax is the draw) or an invalid row.
     if (tid == 0) {
