@@ -312,12 +312,21 @@ def run_ssd(args, rank, world, local_rank):
                 s = sets[i % n_copies]
                 ssd.ssd_verify(s["t"], s["d"], s["tok"], s["u"], w.T, alpha=s["alpha"], fanout_mode=w.fanout_mode,
                                C_coef=w.C, budget=w.budget, cache=True, fallback_seed=w.fallback_seed,
-                               workspace=ws, out=outs[i % n_copies])
+                               workspace=ws, out=outs[i % n_copies], early_exit=args.early_exit)
             kernels = KERNELS_PER_VERIFY
         total_ms, per_step, clocks = time_steps(step, args.steps, args.warmup, dev, world, dist,
                                                 local_rank if rank == 0 else None)
         if world > 1:
             total_ms = max_over_ranks(total_ms, dist, dev)
+        skipped = None
+        if args.early_exit:
+            # target bytes left unread per call, counted on the device over one
+            # pass of the rotating copies (outside the timed region)
+            torch.cuda.synchronize()
+            ws.skipped_bytes()
+            for i in range(n_copies):
+                step(i)
+            skipped = ws.skipped_bytes() / n_copies
         # outcome statistics over every rotating copy's last step
         torch.cuda.synchronize()
         n_acc = np.concatenate([o.n_accepted.cpu().numpy() for o in outs])
@@ -328,10 +337,21 @@ def run_ssd(args, rank, world, local_rank):
                    launches=args.steps * kernels, mean_accepted=float(n_acc.mean()), hit_rate=float(hit.mean()),
                    near_tie_rows=int(((st & ssd.ROW_NEAR_TIE) != 0).sum()), n_copies=n_copies, alg_bytes=alg_bytes,
                    logit_bytes=logit_bytes)
+        if args.early_exit:
+            # the early-exit count: every draft row, the target rows p_0..p_k*
+            # and p_K, from this run's outcomes; the full read beside it
+            s_b = 2 if w.dtype == "bf16" else 4
+            kk = n_acc[n_acc >= 0]
+            p_rows = np.where(kk >= w.K, w.K + 1, kk + 2).mean() if kk.size else w.K + 1
+            ee_logits = w.B * (w.K + p_rows) * w.V * s_b
+            res["alg_bytes"] = int(alg_bytes - logit_bytes + ee_logits)
+            res["early_exit"] = {"alg_bytes_per_launch": res["alg_bytes"], "full_read_bytes_per_launch": alg_bytes,
+                                 "target_bytes_not_read_per_launch": skipped,
+                                 "logit_bytes_read_per_launch": logit_bytes - skipped}
 
         # End to end through the public API from pinned host buffers (rank 0,
         # N=1, default fused step only).
-        if rank == 0 and world == 1 and not args.no_e2e and not args.unfused and not args.sweep:
+        if rank == 0 and world == 1 and not args.no_e2e and not args.unfused and not args.sweep and not args.early_exit:
             def pin(x):
                 if x.dtype == np.uint16:
                     return torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).pin_memory()
@@ -425,6 +445,8 @@ def build_line(args, res, world):
                   f"(together > 2 x 126 MB L2)")
     if args.unfused:
         cfg["step"] = "unfused: fan-out plan, reweight, verify, cache build, cache lookup (one stream)"
+    if args.early_exit:
+        cfg["read_schedule"] = "early exit (ssd_verify_early_exit)"
     line = {
         "metric": METRIC,
         "value": res["rows_per_s"],
@@ -457,6 +479,9 @@ def build_line(args, res, world):
         line["clocks"] = res["clocks"]
     if "e2e" in res:
         line["e2e"] = res["e2e"]
+    if "early_exit" in res:
+        line["early_exit"] = res["early_exit"]
+        line["roofline"]["traffic"] = None
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w, seconds_target=5.0 if args.sweep else 15.0)
     return line
@@ -471,6 +496,7 @@ def main():
     ap.add_argument("--workload", default=None)
     ap.add_argument("--sweep", action="store_true", help="temperature x fan-out mode x C grid, one line each")
     ap.add_argument("--unfused", action="store_true", help="time the five-call unfused step")
+    ap.add_argument("--early-exit", action="store_true", help="the early-exit read schedule (ssd_verify_early_exit)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()

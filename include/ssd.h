@@ -182,8 +182,8 @@ ssd_status ssd_saguaro_reweight(const void* draft_logits, int dtype, int B, int 
                                 int32_t* status, void* workspace, size_t ws_bytes, void* stream);
 
 /*
- * ssd_verify -- the fused verify + cache step, one thread-block cluster per
- * (row, position) streaming that position's target and draft logits once.
+ * ssd_verify -- the fused verify + cache step: CTAs per (row, position,
+ * vocabulary slice) stream that position's target and draft logits once.
  * Lossless verification ([ZH] sections 1-2; [NL] section 2) with Saguaro
  * reweighting: a_j = min(1, p_j(d_j) / q'_j(d_j)); position j is accepted iff
  * u[b,j] < a_j; n_accepted = k* = first rejected j, else K.  The bonus token
@@ -211,6 +211,32 @@ ssd_status ssd_verify(const void* target_logits, const void* draft_logits, const
                       int32_t* n_accepted, int32_t* bonus, int32_t* out_tokens,
                       float* accept_prob, float* residual_mass, const ssd_cache* cache,
                       int32_t* status, void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * ssd_verify_early_exit -- ssd_verify with the early-exit read schedule.
+ * Lossless verification is a prefix test ([ZH] section 1, problem background,
+ * and section 2, basic flow step 2: the drafts are checked in order and the
+ * first rejection ends the accepted prefix), so the outcome (k*, the bonus,
+ * the cache lookup) depends on the target rows p_0..p_{k*} and on p_K (the
+ * source of segment K without draft_next, and of the bonus after full
+ * acceptance) only.  The CTAs of position j (0 < j < K) are scheduled a lag
+ * of rows after those of position j - 1, and a CTA does not read its slice of
+ * p_j when an earlier position of its row is already known to be rejected.
+ * Every draft row q_j is still read (the cache segments need them).
+ *   Arguments and layouts: exactly as ssd_verify.  Outputs: as ssd_verify,
+ *   except that accept_prob[b, j] is NaN for k* < j < K, and that a
+ *   non-finite target row p_j or q'_j(d_j) = 0 at a position k* < j < K does
+ *   not enter status (those rows are not part of the outcome; whether a CTA
+ *   happened to read them never shows in the outputs).  The bytes it did not
+ *   read are counted in the workspace (ssd_read_skipped_bytes).
+ */
+ssd_status ssd_verify_early_exit(const void* target_logits, const void* draft_logits, const void* draft_next,
+                                 int dtype, int B, int K, int V, const int32_t* draft_tokens,
+                                 const float* uniforms, float T, const int32_t* F, const float* alpha,
+                                 int fanout_mode, float C, int budget,
+                                 int32_t* n_accepted, int32_t* bonus, int32_t* out_tokens,
+                                 float* accept_prob, float* residual_mass, const ssd_cache* cache,
+                                 int32_t* status, void* workspace, size_t ws_bytes, void* stream);
 
 /*
  * ssd_verify_noalloc -- ssd_verify with its scratch taken from a static
@@ -319,6 +345,12 @@ size_t ssd_workspace_bytes(int B, int K, int V, int dtype);
  * next use.  Not for the hot path. */
 ssd_status ssd_read_device_error(void* workspace, int B, int K, int V, int dtype, void* stream,
                                  int32_t* out);
+
+/* Reads and clears the workspace's count of target-logit bytes that calls of
+ * ssd_verify_early_exit on it did not read (B, K, V, dtype as laid out),
+ * synchronising `stream`.  A measurement helper, not for the hot path. */
+ssd_status ssd_read_skipped_bytes(void* workspace, int B, int K, int V, int dtype, void* stream,
+                                  uint64_t* out);
 
 const char* ssd_status_string(ssd_status s);
 const char* ssd_version(void);

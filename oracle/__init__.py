@@ -52,7 +52,7 @@ def lib():
             [C.c_int] * 5 + [vp, vp, vp, i32p, f32p, C.c_double, i32p, C.c_double, i32p, C.c_uint64,
                              i32p, C.c_int, C.c_int,
                              i32p, i32p, i32p, f64p, f64p, f64p, f64p, f64p, f64p, i32p, i32p,
-                             u8p, i32p, i32p, i32p, f64p, f64p, f64p, i32p, i32p])
+                             u8p, i32p, i32p, i32p, f64p, f64p, f64p, i32p, i32p, C.c_int])
         L.ssdo_verify_batch.restype = C.c_int
         L.ssdo_reweight_batch.argtypes = (
             [C.c_int] * 5 + [vp, C.c_double, i32p, C.c_double, f32p, i32p, C.c_int, C.c_int,
@@ -162,11 +162,12 @@ def overlap(lp_row, lq_row, T):
 
 
 def verify(target, draft, tokens, uniforms, T, F=None, C_coef=1.0, budget=0, draft_next=None,
-           payload=None, fallback_seed=0, rows=None, n_threads=None, want_phit=False):
+           payload=None, fallback_seed=0, rows=None, n_threads=None, want_phit=False, early_exit=False):
     """Oracle verify + cache step.  target [B,K+1,V], draft [B,K,V] as float32 or
     uint16 bf16 bits; tokens [B,K] int32; uniforms [B,K+1] float32; F [B,K+1]
     int32 or None.  rows: optional subset of batch rows; outputs are indexed by
-    position in that subset."""
+    position in that subset.  early_exit: the early-exit read schedule (target
+    rows p_j past k* other than p_K are not read: no a_j, no flags from them)."""
     target = np.ascontiguousarray(target)
     draft = np.ascontiguousarray(draft)
     B, K1, V = target.shape
@@ -205,7 +206,7 @@ def verify(target, draft, tokens, uniforms, T, F=None, C_coef=1.0, budget=0, dra
         _p(out["hit"], C.c_uint8), _p(out["slot"], C.c_int32), _p(out["next_tokens"], C.c_int32),
         _p(out["status"], C.c_int32), _p(out["accept_margin"], C.c_double),
         _p(out["bonus_margin"], C.c_double), _p(out["p_hit"], C.c_double) if want_phit else None,
-        _p(out["bonus_lo"], C.c_int32), _p(out["bonus_hi"], C.c_int32))
+        _p(out["bonus_lo"], C.c_int32), _p(out["bonus_hi"], C.c_int32), 1 if early_exit else 0)
     if rc != 0:
         raise ValueError("oracle verify rejected its arguments")
     if F is None:

@@ -423,7 +423,35 @@ typedef struct {
   uint8_t* hit; int32_t* slot; int32_t* next_tokens;
   int32_t* status; double* accept_margin; double* bonus_margin; double* p_hit;
   int32_t* bonus_lo; int32_t* bonus_hi;
+  int early_exit;  /* read p_j only for j <= k* and j = K */
 } verify_job;
+
+/* The outputs of an invalid row. */
+static void write_invalid_row(const verify_job* J, int i, int b, int32_t st, int32_t* outt, int32_t* ctok,
+                              int32_t* nxt) {
+  const int K = J->K, V = J->V;
+  J->n_accepted[i] = -1;
+  J->bonus[i] = -1;
+  for (int j = 0; j <= K; ++j) outt[j] = -1;
+  for (int j = 0; j < K; ++j) J->accept_prob[(size_t)i * K + j] = NAN;
+  J->residual_mass[i] = NAN;
+  for (int j = 0; j < K; ++j) {
+    if (J->Z) J->Z[(size_t)i * K + j] = NAN;
+    if (J->QS) J->QS[(size_t)i * K + j] = NAN;
+    if (J->q_lse) J->q_lse[(size_t)i * K + j] = NAN;
+  }
+  if (J->p_lse) for (int j = 0; j <= K; ++j) J->p_lse[(size_t)i * (K + 1) + j] = NAN;
+  if (ctok) for (int s = 0; s < J->budget; ++s) ctok[s] = -1;
+  if (J->hit) J->hit[i] = 0;
+  if (J->slot) J->slot[i] = -1;
+  if (nxt) for (int t = 0; t < K; ++t) nxt[t] = ssdo_fallback_token(J->fallback_seed, b, t, V);
+  J->status[i] = st;
+  if (J->accept_margin) J->accept_margin[i] = INFINITY;
+  if (J->bonus_margin) J->bonus_margin[i] = INFINITY;
+  if (J->p_hit) J->p_hit[i] = NAN;
+  if (J->bonus_lo) J->bonus_lo[i] = -1;
+  if (J->bonus_hi) J->bonus_hi[i] = -1;
+}
 
 static void verify_row(const verify_job* J, int i) {
   const int K = J->K, V = J->V, budget = J->budget;
@@ -432,10 +460,15 @@ static void verify_row(const verify_job* J, int i) {
 
   double** lp = malloc(sizeof(double*) * (size_t)(K + 1));
   double** lq = malloc(sizeof(double*) * (size_t)K);
+  /* A non-finite target row makes the row invalid; with the early-exit read
+   * schedule only the target rows the outcome depends on count: p_j for
+   * j <= k* (decided below) and p_K. */
+  int* pnf = malloc(sizeof(int) * (size_t)(K + 1));
   for (int j = 0; j <= K; ++j) {
     lp[j] = malloc(sizeof(double) * (size_t)V);
     load_row(J->target, J->dtype, (size_t)b * (size_t)(K + 1) + (size_t)j, V, lp[j]);
-    if (!row_finite(lp[j], V)) st |= SSDO_ROW_NONFINITE;
+    pnf[j] = !row_finite(lp[j], V);
+    if (pnf[j] && (!J->early_exit || j == K)) st |= SSDO_ROW_NONFINITE;
   }
   for (int j = 0; j < K; ++j) {
     lq[j] = malloc(sizeof(double) * (size_t)V);
@@ -475,27 +508,7 @@ static void verify_row(const verify_job* J, int i) {
   int32_t* outt = J->out_tokens + (size_t)i * (size_t)(K + 1);
 
   if (st & SSDO_ROW_INVALID) {
-    J->n_accepted[i] = -1;
-    J->bonus[i] = -1;
-    for (int j = 0; j <= K; ++j) outt[j] = -1;
-    for (int j = 0; j < K; ++j) J->accept_prob[(size_t)i * K + j] = NAN;
-    J->residual_mass[i] = NAN;
-    for (int j = 0; j < K; ++j) {
-      if (J->Z) J->Z[(size_t)i * K + j] = NAN;
-      if (J->QS) J->QS[(size_t)i * K + j] = NAN;
-      if (J->q_lse) J->q_lse[(size_t)i * K + j] = NAN;
-    }
-    if (J->p_lse) for (int j = 0; j <= K; ++j) J->p_lse[(size_t)i * (K + 1) + j] = NAN;
-    if (ctok) for (int s = 0; s < budget; ++s) ctok[s] = -1;
-    if (J->hit) J->hit[i] = 0;
-    if (J->slot) J->slot[i] = -1;
-    if (nxt) for (int t = 0; t < K; ++t) nxt[t] = ssdo_fallback_token(J->fallback_seed, b, t, V);
-    J->status[i] = st;
-    if (J->accept_margin) J->accept_margin[i] = INFINITY;
-    if (J->bonus_margin) J->bonus_margin[i] = INFINITY;
-    if (J->p_hit) J->p_hit[i] = NAN;
-    if (J->bonus_lo) J->bonus_lo[i] = -1;
-    if (J->bonus_hi) J->bonus_hi[i] = -1;
+    write_invalid_row(J, i, b, st, outt, ctok, nxt);
     goto done;
   }
 
@@ -510,6 +523,8 @@ static void verify_row(const verify_job* J, int i) {
       if (f > 0) topf_row(k < K ? lq[k] : (ln ? ln : lp[K]), V, f, S[k]);
     }
     double* a = malloc(sizeof(double) * (size_t)K);
+    int* zq = calloc((size_t)K, sizeof(int));
+    int ee_bad = 0;
     int kstar = K, bon = -1;
     int32_t blo = -1, bhi = -1;
     double R = 1.0, amarg = INFINITY, bmarg = INFINITY, phit = NAN;
@@ -522,6 +537,7 @@ static void verify_row(const verify_job* J, int i) {
       for (int j = 0; j < K; ++j) {
         int am = argmax_row(lp[j], V);
         a[j] = (d[j] == am) ? 1.0 : 0.0;
+        if (kstar == K && J->early_exit && pnf[j]) ee_bad = 1;  /* a target row read before k* */
         if (kstar == K && d[j] != am) kstar = j;
         int amq = argmax_row(lq[j], V);
         double qs = 0.0;
@@ -568,14 +584,19 @@ static void verify_row(const verify_job* J, int i) {
           a[j] = ratio < 1.0 ? ratio : 1.0;
         } else {
           a[j] = pd > 0.0 ? 1.0 : 0.0;
-          st |= SSDO_ROW_ZERO_Q;
+          zq[j] = 1;
         }
       }
       for (int j = 0; j < K; ++j) {
+        if (J->early_exit && pnf[j]) { ee_bad = 1; break; }  /* a target row read before k* */
         double mg = fabs((double)u[j] - a[j]);
         if (mg < amarg) amarg = mg;
         if (!((double)u[j] < a[j])) { kstar = j; break; }
       }
+      /* q'(d_j) = 0 is reported for every position, or with the early-exit
+       * schedule for the positions up to k* */
+      for (int j = 0; j < K; ++j)
+        if (zq[j] && (!J->early_exit || j <= kstar)) st |= SSDO_ROW_ZERO_Q;
       /* Bonus token: at a rejection k* < K draw from r = max(0, p - q') / R,
        * R = sum r; if R is 0 draw from p instead (reading); after full
        * acceptance draw from p_K.  One uniform u_K serves every case. */
@@ -624,10 +645,17 @@ static void verify_row(const verify_job* J, int i) {
       free(p); free(qp);
     }
 
+    if (ee_bad) {
+      write_invalid_row(J, i, b, st | SSDO_ROW_NONFINITE, outt, ctok, nxt);
+      for (int k = 0; k <= K; ++k) free(S[k]);
+      free(S); free(a); free(zq);
+      goto done;
+    }
     J->n_accepted[i] = kstar;
     J->bonus[i] = bon;
     for (int j = 0; j <= K; ++j) outt[j] = j < kstar ? d[j] : (j == kstar ? bon : -1);
-    for (int j = 0; j < K; ++j) J->accept_prob[(size_t)i * K + j] = a[j];
+    /* the early-exit schedule reports no a_j past k* (p_j was not read) */
+    for (int j = 0; j < K; ++j) J->accept_prob[(size_t)i * K + j] = (J->early_exit && j > kstar) ? NAN : a[j];
     J->residual_mass[i] = R;
 
     /* Cache build and lookup ([ZH] section 2, basic flow steps 3-4; [NL]
@@ -658,10 +686,11 @@ static void verify_row(const verify_job* J, int i) {
     if (J->bonus_lo) J->bonus_lo[i] = blo;
     if (J->bonus_hi) J->bonus_hi[i] = bhi;
     for (int k = 0; k <= K; ++k) free(S[k]);
-    free(S); free(a);
+    free(S); free(a); free(zq);
   }
 
 done:
+  free(pnf);
   for (int j = 0; j <= K; ++j) free(lp[j]);
   for (int j = 0; j < K; ++j) free(lq[j]);
   free(lp); free(lq); free(ln);
@@ -704,7 +733,7 @@ int ssdo_verify_batch(int dtype, int B, int K, int V, int budget,
                       int32_t* offsets, int32_t* cache_tokens,
                       uint8_t* hit, int32_t* slot, int32_t* next_tokens,
                       int32_t* status, double* accept_margin, double* bonus_margin, double* p_hit,
-                      int32_t* bonus_lo, int32_t* bonus_hi) {
+                      int32_t* bonus_lo, int32_t* bonus_hi, int early_exit) {
   if (B < 0 || K < 1 || V < 1 || !(T >= 0.0) || (F && !(C > 0.0 && C <= 1.0))) return -1;
   if (dtype != SSDO_DTYPE_FP32 && dtype != SSDO_DTYPE_BF16) return -1;
   if (F && (budget < 0 || budget > V)) return -1;
@@ -712,7 +741,7 @@ int ssdo_verify_batch(int dtype, int B, int K, int V, int budget,
                   payload, fallback_seed, rows, rows ? n_rows : B, n_threads,
                   n_accepted, bonus, out_tokens, accept_prob, residual_mass, Z, QS, q_lse, p_lse,
                   offsets, cache_tokens, hit, slot, next_tokens, status, accept_margin,
-                  bonus_margin, p_hit, bonus_lo, bonus_hi};
+                  bonus_margin, p_hit, bonus_lo, bonus_hi, early_exit};
   run_rows(&J, J.n_rows, n_threads, verify_row_thunk);
   return 0;
 }

@@ -79,6 +79,10 @@ def load(build_if_missing: bool = True):
     L.ssd_verify.restype = i32
     L.ssd_verify.argtypes = [vp, vp, vp, i32, i32, i32, i32, vp, vp, f32, vp, vp, i32, f32, i32, vp, vp,
                              vp, vp, vp, C.POINTER(_Cache), vp, vp, sz, vp]
+    L.ssd_verify_early_exit.restype = i32
+    L.ssd_verify_early_exit.argtypes = L.ssd_verify.argtypes
+    L.ssd_read_skipped_bytes.restype = i32
+    L.ssd_read_skipped_bytes.argtypes = [vp, i32, i32, i32, i32, vp, C.POINTER(C.c_uint64)]
     L.ssd_verify_noalloc.restype = i32
     L.ssd_verify_noalloc.argtypes = [vp, vp, vp, i32, i32, i32, i32, vp, vp, f32, vp, vp, i32, f32, i32, vp, vp,
                                      vp, vp, vp, C.POINTER(_Cache), vp, vp]
@@ -178,6 +182,15 @@ class Workspace:
         if out.value != 0:
             self.reset()
         return out.value
+
+    def skipped_bytes(self, stream=None) -> int:
+        """Target-logit bytes that early-exit calls on this workspace did not
+        read since the last query (the counter is cleared)."""
+        out = C.c_uint64(0)
+        _check(load().ssd_read_skipped_bytes(self.ptr(), self.B, self.K, self.V, self.dtype, _stream(stream),
+                                             C.byref(out)),
+               "ssd_read_skipped_bytes")
+        return int(out.value)
 
 
 _default_ws = {}
@@ -311,8 +324,9 @@ def ssd_verify(target: torch.Tensor, draft: torch.Tensor, draft_tokens: torch.Te
                alpha: Optional[torch.Tensor] = None, fanout_mode: int = FANOUT_GEOMETRIC,
                payload: Optional[torch.Tensor] = None, fallback_seed: int = 0,
                workspace: Optional[Workspace] = None, out: Optional[VerifyResult] = None,
-               stream=None) -> VerifyResult:
-    """Fused verify + speculation-cache step on the GPU (see ssd_verify in ssd.h)."""
+               stream=None, early_exit: bool = False) -> VerifyResult:
+    """Fused verify + speculation-cache step on the GPU (see ssd_verify in ssd.h);
+    early_exit=True calls ssd_verify_early_exit (the early-exit read schedule)."""
     B, K1, V = target.shape
     K = K1 - 1
     dev = target.device
@@ -342,15 +356,16 @@ def ssd_verify(target: torch.Tensor, draft: torch.Tensor, draft_tokens: torch.Te
         cstruct = _Cache(out.cache_offsets.data_ptr(), out.cache_tokens.data_ptr(),
                          None if payload is None else payload.data_ptr(), out.hit.data_ptr(),
                          out.slot.data_ptr(), out.next_tokens.data_ptr(), fallback_seed)
+    fn = load().ssd_verify_early_exit if early_exit else load().ssd_verify
     with torch.cuda.device(dev):
-        code = load().ssd_verify(
+        code = fn(
             _ptr(target), _ptr(draft), _ptr(draft_next), dt, B, K, V, _ptr(draft_tokens), _ptr(uniforms),
             float(T), _ptr(F), _ptr(alpha), int(fanout_mode), float(C_coef), int(budget),
             _ptr(out.n_accepted), _ptr(out.bonus),
             _ptr(out.out_tokens), _ptr(out.accept_prob), _ptr(out.residual_mass),
             C.byref(cstruct) if cstruct is not None else None, _ptr(out.status), workspace.ptr(),
             workspace.nbytes, _stream(stream))
-    _check(code, "ssd_verify")
+    _check(code, "ssd_verify_early_exit" if early_exit else "ssd_verify")
     return out
 
 

@@ -148,6 +148,10 @@ struct Plan {
   int n_slices, chunk;
 };
 
+#ifndef SSD_EE_LAG_PCT
+#define SSD_EE_LAG_PCT 300
+#endif
+
 static int sm_count() {
   int dev = 0, n = 148;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
@@ -206,7 +210,7 @@ static cudaError_t prepare_kernel(const void* fn) {
 // counters (zero between calls) and the error word.
 struct WsLayout {
   size_t parts, ustate, dparts, rstate, arrive1, row_arrive, draw_arrive, draw_owner, row_arrive2, rflag, uword, dtot,
-      epoch, k2_done, error, total;
+      epoch, k2_done, error, skipped, total;
   int n_slices;
 };
 
@@ -247,6 +251,8 @@ static WsLayout ws_layout(int B, int K, int V, int dtype) {
   w.epoch = off;       off += sizeof(uint32_t);
   w.k2_done = off;     off += sizeof(int32_t);
   w.error = off;       off += sizeof(int32_t);
+  off = (off + 7) & ~static_cast<size_t>(7);
+  w.skipped = off;     off += sizeof(unsigned long long);
   w.total = up256(off);
   return w;
 }
@@ -268,16 +274,21 @@ static void bind_workspace(Args& a, void* ws, const WsLayout& w) {
   a.epoch = reinterpret_cast<uint32_t*>(base + w.epoch);
   a.k2_done = reinterpret_cast<int32_t*>(base + w.k2_done);
   a.error = reinterpret_cast<int32_t*>(base + w.error);
+  a.skipped = reinterpret_cast<unsigned long long*>(base + w.skipped);
 }
 
 template <typename TIn, bool kAligned, bool kGreedy>
 static ssd_status launch_t(const Args& a, long long units, long long draw_units, cudaStream_t stream) {
-  const void* f1 = reinterpret_cast<const void*>(&ssd_stats_kernel<TIn, kAligned, kGreedy>);
+  const void* f1 = a.early_exit ? reinterpret_cast<const void*>(&ssd_stats_kernel<TIn, kAligned, kGreedy, true>)
+                                 : reinterpret_cast<const void*>(&ssd_stats_kernel<TIn, kAligned, kGreedy, false>);
   const void* f2 = reinterpret_cast<const void*>(&ssd_draw_kernel<TIn, kAligned, kGreedy>);
   if (prepare_kernel(f1) != cudaSuccess || prepare_kernel(f2) != cudaSuccess) return SSD_ERR_CUDA;
   const size_t smem = kRingBytes;  // the ring, and afterwards the merge buffers
-  ssd_stats_kernel<TIn, kAligned, kGreedy>
-      <<<static_cast<unsigned>(stats_grid(a)), kThreads, smem, stream>>>(a);
+  if (a.early_exit)
+    ssd_stats_kernel<TIn, kAligned, kGreedy, true><<<static_cast<unsigned>(stats_grid(a)), kThreads, smem, stream>>>(a);
+  else
+    ssd_stats_kernel<TIn, kAligned, kGreedy, false>
+        <<<static_cast<unsigned>(stats_grid(a)), kThreads, smem, stream>>>(a);
   if (cudaGetLastError() != cudaSuccess) return SSD_ERR_CUDA;
   if (draw_units > 0) {
     // Programmatic dependent launch: the draw kernel may start while the
@@ -387,12 +398,15 @@ ssd_status ssd_cache_lookup(const int32_t* offsets, const int32_t* tokens, int B
   return cudaGetLastError() == cudaSuccess ? SSD_OK : SSD_ERR_CUDA;
 }
 
-ssd_status ssd_verify(const void* target_logits, const void* draft_logits, const void* draft_next, int dtype,
-                      int B, int K, int V, const int32_t* draft_tokens, const float* uniforms, float T,
-                      const int32_t* F, const float* alpha, int fanout_mode, float C, int budget,
-                      int32_t* n_accepted, int32_t* bonus,
-                      int32_t* out_tokens, float* accept_prob, float* residual_mass, const ssd_cache* cache,
-                      int32_t* status, void* workspace, size_t ws_bytes, void* stream) {
+}  // extern "C"
+
+namespace ssd {
+static ssd_status verify_impl(const void* target_logits, const void* draft_logits, const void* draft_next, int dtype,
+                              int B, int K, int V, const int32_t* draft_tokens, const float* uniforms, float T,
+                              const int32_t* F, const float* alpha, int fanout_mode, float C, int budget,
+                              int32_t* n_accepted, int32_t* bonus, int32_t* out_tokens, float* accept_prob,
+                              float* residual_mass, const ssd_cache* cache, int32_t* status, void* workspace,
+                              size_t ws_bytes, void* stream, int early_exit) {
   if (dtype != SSD_DTYPE_BF16 && dtype != SSD_DTYPE_FP32) return SSD_ERR_DTYPE;
   if (B < 0 || K < 1 || K > SSD_MAX_K || V < 1) return SSD_ERR_INVALID_ARG;
   if (!(T >= 0.f) || isinf(T)) return SSD_ERR_INVALID_ARG;
@@ -431,6 +445,15 @@ ssd_status ssd_verify(const void* target_logits, const void* draft_logits, const
   a.units_per_row = K + 1; a.draws = 1;
   a.n_slices = plan.n_slices; a.chunk = plan.chunk;
   if (stats_grid(a) > 0x7FFFFFFFLL) return SSD_ERR_INVALID_ARG;
+  a.early_exit = early_exit;
+  if (early_exit) {
+    // the lag: about the rows whose CTAs are scheduled while one position's
+    // CTAs stream and finalise (SSD_EE_LAG_PCT % of a wave of resident CTAs)
+    const long long per_row = static_cast<long long>(a.units_per_row) * a.n_slices;
+    const long long rows = (static_cast<long long>(SSD_EE_LAG_PCT) * kMinBlocks * sm_count() + 100 * per_row - 1) /
+                           (100 * per_row);
+    a.lag = static_cast<int>(rows < 1 ? 1 : (rows > B ? B : rows));
+  }
   Plan dplan;
   const ssd_status dps = make_plan(V, 2, esize, B, &dplan, kDrawCtaBytes);
   if (dps != SSD_OK) return dps;
@@ -447,6 +470,44 @@ ssd_status ssd_verify(const void* target_logits, const void* draft_logits, const
   bind_workspace(a, workspace, wl);
   const int VE = 16 / esize;
   return launch(a, dtype, V % VE == 0, units, B, static_cast<cudaStream_t>(stream));
+}
+}  // namespace ssd
+
+extern "C" {
+
+ssd_status ssd_verify(const void* target_logits, const void* draft_logits, const void* draft_next, int dtype,
+                      int B, int K, int V, const int32_t* draft_tokens, const float* uniforms, float T,
+                      const int32_t* F, const float* alpha, int fanout_mode, float C, int budget,
+                      int32_t* n_accepted, int32_t* bonus,
+                      int32_t* out_tokens, float* accept_prob, float* residual_mass, const ssd_cache* cache,
+                      int32_t* status, void* workspace, size_t ws_bytes, void* stream) {
+  return verify_impl(target_logits, draft_logits, draft_next, dtype, B, K, V, draft_tokens, uniforms, T, F, alpha,
+                     fanout_mode, C, budget, n_accepted, bonus, out_tokens, accept_prob, residual_mass, cache, status,
+                     workspace, ws_bytes, stream, 0);
+}
+
+ssd_status ssd_verify_early_exit(const void* target_logits, const void* draft_logits, const void* draft_next,
+                                 int dtype, int B, int K, int V, const int32_t* draft_tokens, const float* uniforms,
+                                 float T, const int32_t* F, const float* alpha, int fanout_mode, float C, int budget,
+                                 int32_t* n_accepted, int32_t* bonus, int32_t* out_tokens, float* accept_prob,
+                                 float* residual_mass, const ssd_cache* cache, int32_t* status, void* workspace,
+                                 size_t ws_bytes, void* stream) {
+  return verify_impl(target_logits, draft_logits, draft_next, dtype, B, K, V, draft_tokens, uniforms, T, F, alpha,
+                     fanout_mode, C, budget, n_accepted, bonus, out_tokens, accept_prob, residual_mass, cache, status,
+                     workspace, ws_bytes, stream, 1);
+}
+
+ssd_status ssd_read_skipped_bytes(void* workspace, int B, int K, int V, int dtype, void* stream, uint64_t* out) {
+  if (!workspace || !out || B < 0 || K < 1 || K > SSD_MAX_K || V < 1) return SSD_ERR_INVALID_ARG;
+  if (dtype != SSD_DTYPE_BF16 && dtype != SSD_DTYPE_FP32) return SSD_ERR_DTYPE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  char* word = static_cast<char*>(workspace) + ws_layout(B, K, V, dtype).skipped;
+  unsigned long long v = 0;
+  if (cudaMemcpyAsync(&v, word, sizeof(v), cudaMemcpyDeviceToHost, st) != cudaSuccess) return SSD_ERR_CUDA;
+  if (cudaMemsetAsync(word, 0, sizeof(v), st) != cudaSuccess) return SSD_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return SSD_ERR_CUDA;
+  *out = static_cast<uint64_t>(v);
+  return SSD_OK;
 }
 
 }  // extern "C"

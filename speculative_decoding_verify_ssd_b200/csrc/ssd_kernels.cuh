@@ -102,6 +102,7 @@ struct SlicePart {
   int32_t argP, argQ;             // greedy: lowest id of the slice maximum
   int32_t n_cand, timeout;        // local candidates found; copy timeout
   float xdP, xdQ;                 // logits of the drafted token (the slice that holds it)
+  int32_t pskip, pad2;            // early exit: this slice did not read the target row
   Cand cand[kCandSlice];          // sorted local candidates (at most min(n_cand, F))
 };
 
@@ -147,6 +148,8 @@ struct Args {
   int B, K, V, budget, mode, n_slices, chunk, units_per_row;
   int d_slices, d_chunk;   // kernel 2: slices per drawn row and their length
   int draws;               // kernel 2 runs (verify always; reweight: draft tokens drawn)
+  int early_exit;          // verify: the early-exit read schedule
+  int lag;                 // early exit: rows between the CTAs of position j and j + 1
   float T, C;
   // verify outputs
   int32_t* n_accepted;
@@ -184,6 +187,7 @@ struct Args {
   uint32_t* epoch;         // calls completed on this workspace (kernel 2 advances it)
   int32_t* k2_done;        // kernel 2 CTAs past their wait
   int32_t* error;
+  unsigned long long* skipped;  // early exit: target-row bytes not read
 };
 
 template <typename TIn>
@@ -577,7 +581,7 @@ struct Ring {
   uint32_t* rel;  // [ST] warps done with the stage's current chunk
   const TIn* row0;
   const TIn* row1;
-  int nrows, e0, nvec, nch, n_issued;
+  int nrows, e0, nvec, nch, n_issued;  // row0 may be null with nrows = 2: half 0 is not read
 
   __device__ __forceinline__ unsigned char* stage(int slot, int r) const {
     return buf + (static_cast<size_t>(slot) * 2 + r) * (CV * 16);
@@ -587,19 +591,40 @@ struct Ring {
     const int slot = c % ST;
     const int v0 = c * CV;
     const int nv = min(CV, nvec - v0);
-    mbar_arrive_expect_tx(&full[slot], static_cast<uint32_t>(nv) * 16u * static_cast<uint32_t>(nrows));
-    if constexpr (kEvictFirst) {
-      const uint64_t pol = l2_policy_evict_first();
-      bulk_copy_g2s_hint(stage(slot, 0), row0 + e0 + v0 * VE, static_cast<uint32_t>(nv) * 16u, &full[slot], pol);
-      if (nrows > 1)
-        bulk_copy_g2s_hint(stage(slot, 1), row1 + e0 + v0 * VE, static_cast<uint32_t>(nv) * 16u, &full[slot], pol);
-    } else {
-      bulk_copy_g2s(stage(slot, 0), row0 + e0 + v0 * VE, static_cast<uint32_t>(nv) * 16u, &full[slot]);
-      if (nrows > 1) bulk_copy_g2s(stage(slot, 1), row1 + e0 + v0 * VE, static_cast<uint32_t>(nv) * 16u, &full[slot]);
-    }
+    const int nr = (row0 != nullptr ? 1 : 0) + (nrows > 1 ? 1 : 0);
+    mbar_arrive_expect_tx(&full[slot], static_cast<uint32_t>(nv) * 16u * static_cast<uint32_t>(nr));
+    if (row0 != nullptr) copy_row(slot, 0, row0 + e0 + v0 * VE, nv);
+    if (nrows > 1) copy_row(slot, 1, row1 + e0 + v0 * VE, nv);
     n_issued = c + 1;
   }
-  __device__ __forceinline__ void start(int tid) {
+  __device__ __forceinline__ void copy_row(int slot, int r, const TIn* src, int nv) {
+    if constexpr (kEvictFirst) {
+      bulk_copy_g2s_hint(stage(slot, r), src, static_cast<uint32_t>(nv) * 16u, &full[slot], l2_policy_evict_first());
+    } else {
+      bulk_copy_g2s(stage(slot, r), src, static_cast<uint32_t>(nv) * 16u, &full[slot]);
+    }
+  }
+  // Rows 0 and 1 of the first ST chunks issued separately (two rows only):
+  // row 1 now, its bytes expected without an arrival, so no stage can
+  // complete before issue_first_row0 has decided on row 0.
+  __device__ __forceinline__ void issue_first_row1() {
+    constexpr int VE = 16 / sizeof(TIn);
+    for (int c = 0; c < min(ST, nch); ++c) {
+      const int nv = min(CV, nvec - c * CV);
+      mbar_expect_tx(&full[c], static_cast<uint32_t>(nv) * 16u);
+      copy_row(c, 1, row1 + e0 + c * CV * VE, nv);
+    }
+  }
+  __device__ __forceinline__ void issue_first_row0(bool read0) {
+    constexpr int VE = 16 / sizeof(TIn);
+    for (int c = 0; c < min(ST, nch); ++c) {
+      const int nv = min(CV, nvec - c * CV);
+      mbar_arrive_expect_tx(&full[c], read0 ? static_cast<uint32_t>(nv) * 16u : 0u);
+      if (read0) copy_row(c, 0, row0 + e0 + c * CV * VE, nv);
+    }
+    n_issued = min(ST, nch);
+  }
+  __device__ __forceinline__ void init(int tid) {
     n_issued = 0;
     if (tid == 0) {
       for (int s = 0; s < ST; ++s) {
@@ -609,6 +634,9 @@ struct Ring {
       mbar_init_fence();
     }
     __syncthreads();
+  }
+  __device__ __forceinline__ void start(int tid) {
+    init(tid);
     if (tid == 0)
       for (int c = 0; c < min(ST, nch); ++c) issue(c);
   }
@@ -776,14 +804,14 @@ struct Smem1 {
   int32_t s_F[SSD_MAX_K + 1];
   float tau, MP, SP, MQ, SQ, QS, bx;
   int32_t bi, argP, argQ, n_total, slow, tmo, n_raw, is_last, is_last_row, pad;
-  int32_t Fj, seg_off, plan_bad;
+  int32_t Fj, seg_off, plan_bad, pskip;
   float xdP, xdQ;
   int32_t cand_off[kMaxSlices + 1];
   int32_t cnt[kMaxSlices];
 };
 
 // One statistics CTA: slice `slice` of unit (row b, position j).
-template <typename TIn, bool kAligned, bool kGreedy>
+template <typename TIn, bool kAligned, bool kGreedy, bool kEE>
 __device__ __forceinline__ void stats_cta(const Args& a, int b, int j, int slice, int S, int chunk) {
   constexpr int VE = Elem<TIn>::VE;
   extern __shared__ __align__(128) unsigned char ring_buf[];
@@ -798,9 +826,6 @@ __device__ __forceinline__ void stats_cta(const Args& a, int b, int j, int slice
   const TIn *baseP, *baseQ;
   long long rbP, rbQ;
   unit_rows<TIn>(a, b, j, baseP, rbP, baseQ, rbQ);
-  const bool hasP = baseP != nullptr, hasQ = baseQ != nullptr;
-  const bool srcQ = hasQ;  // the top-F source row: q_j, else p_j
-  const bool has_d = verify && j < K;
 
   // ---- slice [e0, e1) of the rows, vectors of VE elements --------------------------
   const int e0 = slice * chunk;
@@ -812,14 +837,57 @@ __device__ __forceinline__ void stats_cta(const Args& a, int b, int j, int slice
   ring.buf = ring_buf;
   ring.full = sm.full;
   ring.rel = sm.rel;
-  ring.row0 = hasP ? baseP + rbP : baseQ + rbQ;
-  ring.row1 = baseQ + rbQ;
-  ring.nrows = (hasP ? 1 : 0) + (hasQ ? 1 : 0);
   ring.e0 = e0;
   ring.nvec = nvec;
   ring.nch = nch;
-  const int slotP = 0, slotQ = hasP ? 1 : 0;
-  if constexpr (kAligned) ring.start(tid);
+
+  // Early-exit read schedule: the target row p_j (0 < j < K) is not read
+  // once an earlier position of the row is known to be rejected (its unit's
+  // tagged word says so).  Then k* < j, and the outcome does not depend on
+  // p_j; the CTAs of position j are scheduled a lag of rows after those of
+  // position j - 1 so that such rejections are often known in time.  The
+  // draft row's first chunks are in flight while the words are read.
+  bool pskip = false;
+  const bool ee_unit = kEE && verify && j > 0 && j < K;
+  if (ee_unit) {
+    if constexpr (kAligned) {
+      ring.row0 = baseP + rbP;
+      ring.row1 = baseQ + rbQ;
+      ring.nrows = 2;
+      ring.init(tid);
+    }
+    if (warp == 0) {
+      if (kAligned && lane == 0) ring.issue_first_row1();
+      const uint32_t tag = *reinterpret_cast<volatile const uint32_t*>(a.epoch) + 1u;
+      bool rej = false;
+      if (lane < j) {
+        const uint64_t w = ld_acquire_gpu_u64(a.uword + static_cast<long long>(b) * (K + 1) + lane);
+        rej = static_cast<uint32_t>(w >> 32) == tag && ((w >> 16) & 1u) != 0;
+      }
+      rej = __any_sync(0xFFFFFFFFu, rej);
+      if (kAligned && lane == 0) ring.issue_first_row0(!rej);
+      if (lane == 0) sm.pskip = rej ? 1 : 0;
+    }
+    __syncthreads();
+    pskip = sm.pskip != 0;
+    if (pskip) {
+      baseP = nullptr;
+      ring.row0 = nullptr;
+      if (tid == 0) atomicAdd(a.skipped, static_cast<unsigned long long>(n) * sizeof(TIn));
+    }
+  }
+  const bool hasP = baseP != nullptr, hasQ = baseQ != nullptr;
+  const bool srcQ = hasQ;  // the top-F source row: q_j, else p_j
+  const bool has_d = verify && j < K;
+  // ring stage halves: an early-exit unit keeps p in half 0 and q in half 1
+  // whether or not it reads p; otherwise the first row read takes half 0
+  const int slotP = 0, slotQ = (hasP || ee_unit) ? 1 : 0;
+  if (!ee_unit) {
+    ring.row0 = hasP ? baseP + rbP : baseQ + rbQ;
+    ring.row1 = baseQ + rbQ;
+    ring.nrows = (hasP ? 1 : 0) + (hasQ ? 1 : 0);
+    if constexpr (kAligned) ring.start(tid);
+  }
 
   const bool has_plan = a.F != nullptr || a.alpha != nullptr;
   // Warp 0 forms the plan now, while the first chunks are in flight (only the
@@ -972,7 +1040,7 @@ __device__ __forceinline__ void stats_cta(const Args& a, int b, int j, int slice
   // The slice that holds the drafted token reads its two logits for the
   // unit's accept test now (this CTA has just streamed them through L2).
   float xdP = 0.f, xdQ = 0.f;
-  if (!kGreedy && has_d && tid == 0 && d >= e0 && d < e1) {
+  if (!kGreedy && has_d && hasP && tid == 0 && d >= e0 && d < e1) {
     xdP = Elem<TIn>::at(baseP + rbP, d);
     xdQ = Elem<TIn>::at(baseQ + rbQ, d);
   }
@@ -1050,6 +1118,7 @@ __device__ __forceinline__ void stats_cta(const Args& a, int b, int j, int slice
       part->argP = a1; part->argQ = a2;
       part->timeout = tmo;
       part->xdP = xdP; part->xdQ = xdQ;
+      part->pskip = pskip ? 1 : 0;
     }
   } else if (warp == 1) {
     // This slice's threshold: the F-th largest of its thread maxima bounds the
@@ -1166,12 +1235,13 @@ __device__ __forceinline__ void stats_cta(const Args& a, int b, int j, int slice
     // Butterfly over the slices (lanes >= S hold neutral values): bit-identical
     // results whichever CTA finalizes.
     float mp = -INFINITY, sp = 0.f, mq = -INFINITY, sq = 0.f;
-    int ap = INT_MAX, aq = INT_MAX, nc = 0, to = 0;
+    int ap = INT_MAX, aq = INT_MAX, nc = 0, to = 0, ps = 0;
     if (lane < S) {
       mp = __ldcg(&parts[lane].mP); sp = __ldcg(&parts[lane].sP);
       mq = __ldcg(&parts[lane].mQ); sq = __ldcg(&parts[lane].sQ);
       ap = __ldcg(&parts[lane].argP); aq = __ldcg(&parts[lane].argQ);
       nc = __ldcg(&parts[lane].n_cand); to = __ldcg(&parts[lane].timeout);
+      ps = __ldcg(&parts[lane].pskip);
     }
     float xp = 0.f, xq = 0.f;
     if (!kGreedy && has_d && lane < S) {
@@ -1201,6 +1271,7 @@ __device__ __forceinline__ void stats_cta(const Args& a, int b, int j, int slice
     const int total = __shfl_sync(0xFFFFFFFFu, incl, 31);
     const unsigned over = __ballot_sync(0xFFFFFFFFu, nc > kCandCap || (nc > kCandSlice && Fj > kCandSlice));
     const unsigned anyto = __ballot_sync(0xFFFFFFFFu, to != 0);
+    const unsigned anyskip = __ballot_sync(0xFFFFFFFFu, ps != 0);
     if (lane < S) {
       sm.cand_off[lane] = incl - cnt;
       sm.cnt[lane] = cnt;
@@ -1212,22 +1283,29 @@ __device__ __forceinline__ void stats_cta(const Args& a, int b, int j, int slice
       sm.n_total = total;
       sm.tmo = anyto ? 1 : 0;
       sm.slow = over || total > kGatherCap || total < Fj;
+      sm.pskip = anyskip ? 1 : 0;
     }
   }
   __syncthreads();
   const float MP = sm.MP, MQ = sm.MQ, SP = sm.SP, SQ = sm.SQ;
   if (sm.tmo || !arrivals_ok) flags |= kFlagTimeout;
-  // a non-finite target row is kept apart (pflags): the row decision may
-  // count it only for the positions the outcome depends on
-  const int pflags = (hasP && !(MP > -INFINITY && MP < INFINITY)) ? SSD_ROW_NONFINITE : 0;
+  // Early exit: when a slice skipped p_j, position j lies past k* and its
+  // accept test is not taken (a_j is not reported).
+  const bool p_read = verify && sm.pskip == 0;
+  // a non-finite target row and q'(d_j) = 0 are kept apart (pflags): with the
+  // early-exit schedule the row counts them only up to k*
+  int pflags = (p_read && !(MP > -INFINITY && MP < INFINITY)) ? SSD_ROW_NONFINITE : 0;
   if (hasQ && !(MQ > -INFINITY && MQ < INFINITY)) flags |= SSD_ROW_NONFINITE;
   const bool valid = ((flags | pflags) & SSD_ROW_INVALID) == 0;
-  const bool slow = want_topf && valid && (!one_round || sm.slow != 0);
+  // the top-F set, Z and the cache segment depend on the source row only (q_j,
+  // or p_K for segment K): a bad target row past k* must not void them
+  const bool valid_src = ((flags | (srcQ ? 0 : pflags)) & SSD_ROW_INVALID) == 0;
+  const bool slow = want_topf && valid_src && (!one_round || sm.slow != 0);
   Cand* sel = gbuf + kGatherCap;
   const float nmP = -MP * cT, nmQ = -MQ * cT;
 
   // ---- exact top-F: global ranks by binary search in the sorted slice lists --------
-  if (want_topf && valid && !slow) {
+  if (want_topf && valid_src && !slow) {
     for (int i = tid; i < S * cap; i += kThreads) {
       const int c = i / cap, r0 = i - c * cap;
       if (r0 >= sm.cnt[c]) continue;
@@ -1257,7 +1335,7 @@ __device__ __forceinline__ void stats_cta(const Args& a, int b, int j, int slice
   // Q_S in a fixed order, and the top-F boundary.
   if (warp == 0) {
     float qs = 0.f;
-    if (want_topf && valid) {
+    if (want_topf && valid_src) {
       if constexpr (!kGreedy) {
         for (int i = lane; i < Fj; i += 32) qs += ex2(fmaf(sel[i].x, cT, srcQ ? nmQ : nmP));
       }
@@ -1265,8 +1343,8 @@ __device__ __forceinline__ void stats_cta(const Args& a, int b, int j, int slice
     qs = warp_sum(qs);
     if (lane == 0) {
       sm.QS = qs;
-      sm.bx = (want_topf && valid) ? sel[Fj - 1].x : INFINITY;
-      sm.bi = (want_topf && valid) ? sel[Fj - 1].idx : -1;
+      sm.bx = (want_topf && valid_src) ? sel[Fj - 1].x : INFINITY;
+      sm.bi = (want_topf && valid_src) ? sel[Fj - 1].idx : -1;
     }
   }
   __syncthreads();
@@ -1274,12 +1352,15 @@ __device__ __forceinline__ void stats_cta(const Args& a, int b, int j, int slice
   // ---- Saguaro normaliser and the accept test --------------------------------------
   const float C = a.C;
   float Z = 1.f;
-  if (!kGreedy && want_topf && valid) Z = 1.f - (1.f - C) * (sm.QS / (srcQ ? SQ : SP));
+  if (!kGreedy && want_topf && valid_src) Z = 1.f - (1.f - C) * (sm.QS / (srcQ ? SQ : SP));
   const float bx = sm.bx;
   const int bi = sm.bi;
   float acc = 0.f, amargin = INFINITY;
   int rejected = 0;
-  if (has_d && valid) {
+  if (has_d && valid && !p_read) {
+    acc = __int_as_float(0x7FC00000);
+    rejected = 1;
+  } else if (has_d && valid) {
     if constexpr (kGreedy) {
       acc = (d == sm.argP) ? 1.f : 0.f;
       rejected = d != sm.argP;
@@ -1293,7 +1374,7 @@ __device__ __forceinline__ void stats_cta(const Args& a, int b, int j, int slice
         acc = fminf(1.f, pd / qpd);
       } else {
         acc = pd > 0.f ? 1.f : 0.f;
-        flags |= SSD_ROW_ZERO_Q;
+        pflags |= SSD_ROW_ZERO_Q;
       }
       rejected = !(u_self < acc);
       amargin = fabsf(u_self - acc);
@@ -1308,7 +1389,7 @@ __device__ __forceinline__ void stats_cta(const Args& a, int b, int j, int slice
     segdst = a.topf_tokens + static_cast<long long>(b) * a.budget + seg_off;
   }
   if (segdst && has_plan)
-    for (int i = tid; i < Fj; i += kThreads) segdst[i] = valid ? sel[i].idx : -1;
+    for (int i = tid; i < Fj; i += kThreads) segdst[i] = valid_src ? sel[i].idx : -1;
   if (tid == 0) {
     if (verify && j < K) a.accept_prob[static_cast<long long>(b) * K + j] = valid ? acc : __int_as_float(0x7FC00000);
     if (!verify && j < K) {
@@ -1435,19 +1516,67 @@ __device__ __forceinline__ void stats_cta(const Args& a, int b, int j, int slice
   }
 }
 
+// The early-exit order of the units: unit (b, j) has the key b for j = 0 and
+// j = K, and b + j * lag for 0 < j < K; units are taken by (key, j), so the
+// CTAs of position j come a lag of rows after those of position j - 1.
+// One warp maps order index o to (b, j): a 32-way search for the key (the
+// count of units below a key is monotone in the key), then the rank among
+// the units of that key.
+__device__ __noinline__ void lagged_unit_warp(int o, int B, int K, int lag, int lane, int& b, int& j) {
+  auto below = [&](int c) {  // units whose key is below c
+    long long cnt = 2LL * min(max(c, 0), B);
+    for (int jj = 1; jj < K; ++jj) cnt += min(max(c - jj * lag, 0), B);
+    return cnt;
+  };
+  auto off = [&](int jj) { return (jj == 0 || jj == K) ? 0 : jj * lag; };
+  int lo = 0, hi = B + (K - 1) * lag;  // the key lies in [lo, hi); below(lo) <= o
+  while (hi - lo > 1) {
+    const int step = (hi - lo + 31) / 32;
+    const int c = lo + step * lane;
+    const unsigned ok = __ballot_sync(0xFFFFFFFFu, c < hi && below(c) <= o);
+    const int last = 31 - __clz(ok);  // lane 0 (c = lo) always qualifies
+    hi = min(hi, lo + step * (last + 1));
+    lo += step * last;
+  }
+  const int r = static_cast<int>(o - below(lo));
+  const int bb = lo - off(lane);
+  const unsigned has = __ballot_sync(0xFFFFFFFFu, lane <= K && bb >= 0 && bb < B);
+  if (r < __popc(has)) {  // the lane holding the r-th unit of the key
+    const bool mine = ((has >> lane) & 1u) && __popc(has & ((1u << lane) - 1u)) == r;
+    j = __ffs(__ballot_sync(0xFFFFFFFFu, mine)) - 1;
+  } else {
+    j = 32;  // K = 32: unit 32 sits past the warp's lanes, at key b
+  }
+  b = lo - off(j);
+}
+
 // Kernel 1 of the two-kernel form (the draft side's ssd_saguaro_reweight):
 // one CTA per (unit, slice), rows in order so that rows are decided one
 // after another.
-template <typename TIn, bool kAligned, bool kGreedy>
+template <typename TIn, bool kAligned, bool kGreedy, bool kEE>
 __global__ void __launch_bounds__(kThreads, kMinBlocks) ssd_stats_kernel(const __grid_constant__ Args a) {
   const int S = a.n_slices;
   const int order = blockIdx.x / S, slice = blockIdx.x % S;
   const int upr = a.units_per_row;
-  const int b = order / upr, j = order % upr;
+  int b = order / upr, j = order % upr;
+  if constexpr (kEE) {
+    __shared__ int s_unit[2];
+    if (threadIdx.x < 32) {
+      int bb, jj;
+      lagged_unit_warp(order, a.B, a.K, a.lag, static_cast<int>(threadIdx.x), bb, jj);
+      if (threadIdx.x == 0) {
+        s_unit[0] = bb;
+        s_unit[1] = jj;
+      }
+    }
+    __syncthreads();
+    b = s_unit[0];
+    j = s_unit[1];
+  }
   // kernel 2 may be scheduled once every CTA of this grid has started; it
   // waits for each of its units' records on its own
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-  stats_cta<TIn, kAligned, kGreedy>(a, b, j, slice, S, a.chunk);
+  stats_cta<TIn, kAligned, kGreedy, kEE>(a, b, j, slice, S, a.chunk);
 }
 
 // Shared memory of kernel 2.
@@ -1592,10 +1721,11 @@ __device__ __forceinline__ void draw_cta(const Args& a, int du, int slice) {
       const uint32_t lo0 = static_cast<uint32_t>(w0), lo1 = static_cast<uint32_t>(w1);
       const unsigned rm = __ballot_sync(0xFFFFFFFFu, lane < K && ((lo0 >> 16) & 1u));
       const int kstar = rm ? __ffs(rm) - 1 : K;
-      // flags of every unit; a non-finite target row, a near-tie accept test
-      // only up to k*
+      // flags of every unit; a near-tie accept test only up to k*; with the
+      // early-exit schedule a non-finite target row and q'(d) = 0 only up to
+      // k* and at K (unit 32 is K itself)
       uint32_t f = (lo0 | lo1) & 0xFFu;
-      f |= (lo0 >> 8) & 0xFFu;
+      if (!a.early_exit || lane <= kstar || lane == K) f |= (lo0 >> 8) & 0xFFu;
       f |= (lo1 >> 8) & 0xFFu;
       if (lane <= kstar && ((lo0 >> 17) & 1u)) f |= SSD_ROW_NEAR_TIE;
       f = __reduce_or_sync(0xFFFFFFFFu, f);
@@ -2043,6 +2173,9 @@ __device__ __forceinline__ void draw_cta(const Args& a, int du, int slice) {
   }
   if (invalid)
     for (int k = tid; k < K; k += kThreads) a.accept_prob[static_cast<long long>(b) * K + k] = __int_as_float(0x7FC00000);
+  else if (a.early_exit)  // no a_j past k*: p_j is not part of the outcome
+    for (int k = kstar + 1 + tid; k < K; k += kThreads)
+      a.accept_prob[static_cast<long long>(b) * K + k] = __int_as_float(0x7FC00000);
   if (a.c_tokens) {
     const bool pbad = (fl & SSD_ROW_BAD_PLAN) != 0;
     if (tid == 0) {

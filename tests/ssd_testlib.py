@@ -87,7 +87,7 @@ class Case:
         self.payload = None
         self.with_F = True
 
-    def run_gpu(self, cache=True, with_F=True, payload=None):
+    def run_gpu(self, cache=True, with_F=True, payload=None, early_exit=False):
         w, g = self.w, self.g
         self.payload = payload
         self.with_F = with_F
@@ -98,18 +98,18 @@ class Case:
                            F=to_dev(self.F) if with_F else None, C_coef=w.C, budget=w.budget,
                            draft_next=dn, cache=cache and with_F,
                            payload=to_dev(payload) if payload is not None else None,
-                           fallback_seed=w.fallback_seed)
+                           fallback_seed=w.fallback_seed, early_exit=early_exit)
         torch.cuda.synchronize()
         return {k: (v.cpu().numpy() if isinstance(v, torch.Tensor) else v) for k, v in r.__dict__.items()}
 
-    def run_oracle(self, with_F=True, payload=None, want_phit=False):
+    def run_oracle(self, with_F=True, payload=None, want_phit=False, early_exit=False):
         w, g = self.w, self.g
         self.with_F = with_F
         self.payload = payload
         return oracle.verify(g["target"], g["draft"], self.tokens, g["uniforms"], w.T,
                              F=self.F if with_F else None, C_coef=w.C, budget=w.budget,
                              draft_next=self.draft_next, payload=payload, fallback_seed=w.fallback_seed,
-                             rows=self.rows, want_phit=want_phit)
+                             rows=self.rows, want_phit=want_phit, early_exit=early_exit)
 
 
 NEAR_TIE = 1e-5
@@ -165,7 +165,7 @@ def _outcome_ok(gk, gb, grm, o, i):
     return abs(float(grm) - o["residual_mass"][i]) < PROB_ATOL
 
 
-def compare(case, gpu, orc, with_cache=True):
+def compare(case, gpu, orc, with_cache=True, early_exit=False):
     """Element-by-element comparison; returns the number of near-tie rows.
 
     Rows whose every decision margin is at least 1e-5 are bit-exact.  A row
@@ -175,7 +175,9 @@ def compare(case, gpu, orc, with_cache=True):
     the oracle's or the oracle's outcome with that one decision flipped.  The
     cache keys are checked bit for bit on every row, and hit / slot / next
     tokens must be what a brute-force lookup of the GPU's own (k*, bonus) in
-    the oracle's cache gives."""
+    the oracle's cache gives.  early_exit: the oracle ran the early-exit
+    schedule (no a_j past k*); a_j is compared where both report one, and a
+    row with the oracle's own k* must report none past it."""
     rows = np.arange(case.w.B) if case.rows is None else np.asarray(case.rows)
     K = case.K
     st_o = orc["status"]
@@ -186,9 +188,17 @@ def compare(case, gpu, orc, with_cache=True):
     ap_g, ap_o = gpu["accept_prob"][rows], orc["accept_prob"]
     assert np.all(np.isnan(ap_g[invalid])), "invalid rows must carry NaN accept_prob"
     v = ~invalid
-    if v.any():
+    if v.any() and not early_exit:
         err = np.max(np.abs(ap_g[v].astype(np.float64) - ap_o[v]))
         assert err < PROB_ATOL, f"accept_prob max err {err}"
+    if v.any() and early_exit:
+        both = v[:, None] & np.isfinite(ap_o) & np.isfinite(ap_g)
+        if both.any():
+            err = np.max(np.abs(ap_g[both].astype(np.float64) - ap_o[both]))
+            assert err < PROB_ATOL, f"accept_prob max err {err}"
+        same_k = v & (gpu["n_accepted"][rows] == orc["n_accepted"])
+        np.testing.assert_array_equal(np.isnan(ap_g[same_k]), np.isnan(ap_o[same_k]),
+                                      err_msg="early exit: a_j reported past k*, or missing before it")
     np.testing.assert_array_equal(gpu["n_accepted"][rows][invalid], -1)
     np.testing.assert_array_equal(gpu["bonus"][rows][invalid], -1)
     near = 0
@@ -229,8 +239,9 @@ def compare(case, gpu, orc, with_cache=True):
     return near
 
 
-def check_row_properties(case, gpu, with_cache=True):
-    """Properties that hold for every row at any size."""
+def check_row_properties(case, gpu, with_cache=True, early_exit=False):
+    """Properties that hold for every row at any size.  early_exit: a_j is
+    reported up to k* only."""
     K, V = case.K, case.w.V
     st = gpu["status"]
     valid = (st & ssd.ROW_INVALID) == 0
@@ -239,6 +250,10 @@ def check_row_properties(case, gpu, with_cache=True):
     bon = gpu["bonus"]
     assert np.all((bon[valid] >= 0) & (bon[valid] < V))
     ap = gpu["accept_prob"][valid]
+    if early_exit:
+        past = np.arange(K)[None, :] > k[valid][:, None]
+        assert np.all(np.isnan(ap[past])), "early exit: a_j reported past k*"
+        ap = ap[~past]
     assert np.all((ap >= 0) & (ap <= 1))
     for b in np.nonzero(valid)[0]:
         kk = k[b]

@@ -810,3 +810,96 @@ def test_fallback_small_batches_primary_large_batches_fast():
     batches switch to the fast one."""
     bs, choice = oracle.fallback_bstar(0.95, 0.7, 6, 20.0, 2.0, 0.05, 1.0, 4096)
     assert choice[0] == 0 and 1 < bs <= 4096 and choice[-1] == 1
+
+
+# ---------------------------------------------------------------------------
+# Early-exit read schedule: the outcome depends on p_0..p_{k*} and p_K only.
+# ---------------------------------------------------------------------------
+def _ee_batch(seed, B=24, K=5, V=64, T=1.0):
+    rng = np.random.default_rng(seed)
+    lp = rng.normal(0.0, 1.5, (B, K + 1, V)).astype(np.float32)
+    lq = (lp[:, :K] + rng.normal(0.0, 1.2, (B, K, V))).astype(np.float32)
+    D = rng.integers(0, V, (B, K)).astype(np.int32)
+    if T == 0.0:  # greedy: row i drafts the target argmax at its first i mod (K+1) positions
+        for i in range(B):
+            for j in range(i % (K + 1)):
+                D[i, j] = int(np.argmax(lp[i, j]))
+    U = synth.uniforms(seed + 7, B, K + 1, 0)
+    F = np.tile(oracle.fanout_plan(0.6, K, 8), (B, 1))
+    return lp, lq, D, U, F
+
+
+def _verify(lp, lq, D, U, F, T, early_exit):
+    return oracle.verify(lp, lq, D, U, T, F=F, C_coef=0.5, budget=8, fallback_seed=5, early_exit=early_exit)
+
+
+@pytest.mark.parametrize("T", [1.0, 0.0])
+def test_early_exit_outcome_equals_full_read(T):
+    lp, lq, D, U, F = _ee_batch(11, T=T)
+    full = _verify(lp, lq, D, U, F, T, False)
+    ee = _verify(lp, lq, D, U, F, T, True)
+    K = D.shape[1]
+    assert len(set(full["n_accepted"].tolist())) > 2  # rows stop at several positions
+    for k in ("n_accepted", "bonus", "out_tokens", "offsets", "cache_tokens", "hit", "slot", "next_tokens",
+              "bonus_lo", "bonus_hi"):
+        np.testing.assert_array_equal(ee[k], full[k], err_msg=k)
+    np.testing.assert_array_equal(ee["residual_mass"], full["residual_mass"])
+    np.testing.assert_array_equal(ee["accept_margin"], full["accept_margin"])
+    # a_j up to k*, nothing past it
+    for i, ks in enumerate(full["n_accepted"]):
+        np.testing.assert_array_equal(ee["accept_prob"][i, :min(ks + 1, K)], full["accept_prob"][i, :min(ks + 1, K)])
+        assert np.all(np.isnan(ee["accept_prob"][i, ks + 1:]))
+    # the only status difference allowed is q'(d) = 0 past k*
+    assert np.all((ee["status"] ^ full["status"]) & ~oracle.ROW_ZERO_Q == 0)
+
+
+@pytest.mark.parametrize("T", [1.0, 0.0])
+def test_early_exit_ignores_rows_it_does_not_read(T):
+    """Target rows past k* (other than p_K) can hold anything, NaN included:
+    the early-exit outcome equals the full read of the same batch with those
+    rows replaced by finite ones; a NaN at or before k*, or in p_K, still
+    makes the row invalid."""
+    lp, lq, D, U, F = _ee_batch(12, T=T)
+    base = _verify(lp, lq, D, U, F, T, False)
+    K = D.shape[1]
+    junk = lp.copy()
+    unread = np.zeros(lp.shape[:2], bool)
+    for i, ks in enumerate(base["n_accepted"]):
+        for j in range(ks + 1, K):
+            junk[i, j, :] = np.nan if (i + j) % 2 else 1e30
+            unread[i, j] = True
+    assert unread.sum() > 10
+    ee = _verify(junk, lq, D, U, F, T, True)
+    for k in ("n_accepted", "bonus", "out_tokens", "cache_tokens", "hit", "slot", "next_tokens"):
+        np.testing.assert_array_equal(ee[k], base[k], err_msg=k)
+    assert np.all(ee["status"] & oracle.ROW_INVALID == 0)
+    full_junk = _verify(junk, lq, D, U, F, T, False)
+    nan_rows = np.array([np.isnan(junk[i]).any() for i in range(junk.shape[0])])
+    assert np.all(full_junk["status"][nan_rows] & oracle.ROW_NONFINITE)  # the full read sees them
+    # a NaN in a row that is read: p_{k*} or p_K
+    bad = lp.copy()
+    i0 = int(np.argmax(base["n_accepted"] < K))
+    bad[i0, base["n_accepted"][i0], 3] = np.nan
+    bad[i0 + 1, K, 0] = np.nan
+    ee_bad = _verify(bad, lq, D, U, F, T, True)
+    assert ee_bad["status"][i0] & oracle.ROW_NONFINITE and ee_bad["n_accepted"][i0] == -1
+    assert ee_bad["status"][i0 + 1] & oracle.ROW_NONFINITE and ee_bad["n_accepted"][i0 + 1] == -1
+
+
+def test_early_exit_zero_q_only_up_to_k_star():
+    """q'(d_j) = 0 (a draft token outside the reweighted support) is reported
+    by the full read at any position, by the early-exit read only up to k*."""
+    rng = np.random.default_rng(13)
+    B, K, V = 1, 3, 16
+    lp = rng.normal(0.0, 1.0, (B, K + 1, V)).astype(np.float32)
+    lq = lp[:, :K].copy()
+    D = np.array([[2, 5, 7]], np.int32)
+    lq[0, 2, 7] = -np.inf  # q_2(d_2) = 0
+    U = np.array([[0.999, 0.5, 0.5, 0.5]], np.float32)  # position 0 rejects unless a_0 = 1
+    lp[0, 0, 2] = -8.0  # small p_0(d_0): a_0 < 0.999
+    F = np.array([[1, 1, 1, 1]], np.int32)
+    full = oracle.verify(lp, lq, D, U, 1.0, F=F, C_coef=1.0, budget=4, early_exit=False)
+    ee = oracle.verify(lp, lq, D, U, 1.0, F=F, C_coef=1.0, budget=4, early_exit=True)
+    assert full["n_accepted"][0] == 0 and ee["n_accepted"][0] == 0
+    assert full["status"][0] & oracle.ROW_ZERO_Q
+    assert not ee["status"][0] & oracle.ROW_ZERO_Q
