@@ -138,9 +138,9 @@ __device__ __forceinline__ void st_release_gpu_u64(uint64_t* p, uint64_t v) {
 // Bounded wait for a 64-bit word whose high half is a tag: true (and the
 // word in *out) once the high half equals `tag`; false after `limit_ns`.
 __device__ __forceinline__ bool wait_tagged(const uint64_t* word, uint32_t tag, unsigned long long limit_ns,
-                                            uint64_t* out) {
+                                            uint64_t* out, uint32_t max_sleep_ns = 256) {
   const unsigned long long t0 = global_ns();
-  uint32_t sleep_ns = 64;
+  uint32_t sleep_ns = 32;
   for (uint32_t i = 0; i < 50000000u; ++i) {
     const uint64_t v = ld_acquire_gpu_u64(word);
     if (static_cast<uint32_t>(v >> 32) == tag) {
@@ -149,7 +149,7 @@ __device__ __forceinline__ bool wait_tagged(const uint64_t* word, uint32_t tag, 
     }
     if (global_ns() - t0 > limit_ns) return false;
     __nanosleep(sleep_ns);
-    if (sleep_ns < 256) sleep_ns <<= 1;
+    if (sleep_ns < max_sleep_ns) sleep_ns <<= 1;
   }
   return false;
 }

@@ -48,6 +48,9 @@ namespace ssd {
 
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
+#ifndef SSD_STATS_EVICT_FIRST
+#define SSD_STATS_EVICT_FIRST 1
+#endif
 #ifndef SSD_MIN_BLOCKS
 #define SSD_MIN_BLOCKS 5
 #endif
@@ -804,8 +807,9 @@ struct Smem1 {
   int32_t s_F[SSD_MAX_K + 1];
   float tau, MP, SP, MQ, SQ, QS, bx;
   int32_t bi, argP, argQ, n_total, slow, tmo, n_raw, is_last, is_last_row, pad;
-  int32_t Fj, seg_off, plan_bad, pskip;
-  float xdP, xdQ;
+  int32_t Fj, seg_off, plan_bad, pskip, d_tok;
+  uint32_t epoch0;
+  float xdP, xdQ, xdP0, xdQ0;
   int32_t cand_off[kMaxSlices + 1];
   int32_t cnt[kMaxSlices];
 };
@@ -833,7 +837,7 @@ __device__ __forceinline__ void stats_cta(const Args& a, int b, int j, int slice
   const int n = max(0, e1 - e0);
   const int nvec = (n + VE - 1) / VE;
   const int nch = (nvec + kStatsChunkVecs - 1) / kStatsChunkVecs;
-  Ring<TIn, kStatsChunkVecs, kStatsStages, true> ring;  // read once: first out of L2
+  Ring<TIn, kStatsChunkVecs, kStatsStages, SSD_STATS_EVICT_FIRST != 0> ring;  // read once: first out of L2
   ring.buf = ring_buf;
   ring.full = sm.full;
   ring.rel = sm.rel;
@@ -879,6 +883,22 @@ __device__ __forceinline__ void stats_cta(const Args& a, int b, int j, int slice
   const bool hasP = baseP != nullptr, hasQ = baseQ != nullptr;
   const bool srcQ = hasQ;  // the top-F source row: q_j, else p_j
   const bool has_d = verify && j < K;
+  // Thread 0 requests the call's epoch (it cannot advance before every unit
+  // of this call has published), the drafted token and, in the slice that
+  // holds it, its two logits for the unit's accept test; they land in
+  // shared memory while the first chunks are in flight, so the epilogue
+  // needs no round trip for them.
+  uint32_t epoch_ld = 0;
+  int d_ld = -1;
+  float xdP_ld = 0.f, xdQ_ld = 0.f;
+  if (tid == 0) {
+    epoch_ld = *reinterpret_cast<volatile const uint32_t*>(a.epoch);
+    if (has_d) d_ld = __ldg(a.tokens + static_cast<long long>(b) * K + j);
+    if (!kGreedy && has_d && hasP && d_ld >= e0 && d_ld < e1) {
+      xdP_ld = Elem<TIn>::at(baseP + rbP, d_ld);
+      xdQ_ld = Elem<TIn>::at(baseQ + rbQ, d_ld);
+    }
+  }
   // ring stage halves: an early-exit unit keeps p in half 0 and q in half 1
   // whether or not it reads p; otherwise the first row read takes half 0
   const int slotP = 0, slotQ = (hasP || ee_unit) ? 1 : 0;
@@ -887,6 +907,12 @@ __device__ __forceinline__ void stats_cta(const Args& a, int b, int j, int slice
     ring.row1 = baseQ + rbQ;
     ring.nrows = (hasP ? 1 : 0) + (hasQ ? 1 : 0);
     if constexpr (kAligned) ring.start(tid);
+  }
+  if (tid == 0) {
+    sm.epoch0 = epoch_ld;
+    sm.d_tok = d_ld;
+    sm.xdP0 = xdP_ld;
+    sm.xdQ0 = xdQ_ld;
   }
 
   const bool has_plan = a.F != nullptr || a.alpha != nullptr;
@@ -934,10 +960,6 @@ __device__ __forceinline__ void stats_cta(const Args& a, int b, int j, int slice
   }
   int flags = 0, d = -1;
   float u_self = 0.f;
-  if (has_d) {
-    d = __ldg(a.tokens + static_cast<long long>(b) * K + j);
-    if (d < 0 || d >= V) flags |= SSD_ROW_BAD_TOKEN;
-  }
   if (verify) {
     u_self = __ldg(a.uniforms + static_cast<long long>(b) * (K + 1) + j);
     if (!(u_self >= 0.f && u_self < 1.f)) flags |= SSD_ROW_BAD_UNIFORM;
@@ -1037,13 +1059,6 @@ __device__ __forceinline__ void stats_cta(const Args& a, int b, int j, int slice
     f2_unpack(sQ2, lo, hi);
     sQ = lo + hi;
   }
-  // The slice that holds the drafted token reads its two logits for the
-  // unit's accept test now (this CTA has just streamed them through L2).
-  float xdP = 0.f, xdQ = 0.f;
-  if (!kGreedy && has_d && hasP && tid == 0 && d >= e0 && d < e1) {
-    xdP = Elem<TIn>::at(baseP + rbP, d);
-    xdQ = Elem<TIn>::at(baseQ + rbQ, d);
-  }
   sm.gmax[tid] = vm1;
   if (tid == 0) sm.n_raw = 0;
 
@@ -1085,6 +1100,10 @@ __device__ __forceinline__ void stats_cta(const Args& a, int b, int j, int slice
     }
   }
   tmo = __syncthreads_or(tmo);
+  if (has_d) {
+    d = sm.d_tok;
+    if (d < 0 || d >= V) flags |= SSD_ROW_BAD_TOKEN;
+  }
   int Fj = 0, seg_off = 0, plan_bad = 0;
   if (has_plan) {
     plan_bad = sm.plan_bad;
@@ -1117,7 +1136,7 @@ __device__ __forceinline__ void stats_cta(const Args& a, int b, int j, int slice
       part->mQ = m2; part->sQ = kGreedy ? 0.f : s2;
       part->argP = a1; part->argQ = a2;
       part->timeout = tmo;
-      part->xdP = xdP; part->xdQ = xdQ;
+      part->xdP = sm.xdP0; part->xdQ = sm.xdQ0;
       part->pskip = pskip ? 1 : 0;
     }
   } else if (warp == 1) {
@@ -1413,7 +1432,7 @@ __device__ __forceinline__ void stats_cta(const Args& a, int b, int j, int slice
     // row's K+1 words and take the decision themselves (k* = the first
     // rejected position), so no CTA here waits for the rest of the row.
     if (tid == 0) {
-      const uint64_t tag = *reinterpret_cast<volatile uint32_t*>(a.epoch) + 1u;
+      const uint64_t tag = sm.epoch0 + 1u;
       const uint32_t lo = static_cast<uint32_t>(flags & 0xFF) | static_cast<uint32_t>(pflags & 0xFF) << 8 |
                           static_cast<uint32_t>(rejected ? 1 : 0) << 16 |
                           static_cast<uint32_t>(amargin < kNearTie ? 1 : 0) << 17;
@@ -1715,7 +1734,7 @@ __device__ __forceinline__ void draw_cta(const Args& a, int du, int slice) {
       const uint64_t* uw = a.uword + static_cast<long long>(du) * upr;
       uint64_t w0 = 0, w1 = 0;
       bool ok = true;
-      if (lane < upr) ok = wait_tagged(uw + lane, epoch + 1u, kDepWaitNs, &w0);
+      if (lane < upr) ok = wait_tagged(uw + lane, epoch + 1u, kDepWaitNs, &w0, 128u);
       if (lane + 32 < upr) ok = wait_tagged(uw + lane + 32, epoch + 1u, kDepWaitNs, &w1) && ok;
       const bool all_ok = __all_sync(0xFFFFFFFFu, ok);
       const uint32_t lo0 = static_cast<uint32_t>(w0), lo1 = static_cast<uint32_t>(w1);
@@ -2033,7 +2052,7 @@ __device__ __forceinline__ void draw_cta(const Args& a, int du, int slice) {
         }
         uint64_t wv = 0;
         bool ok = true;
-        if (lane < S) ok = wait_tagged(dtot + lane, tag, kDepWaitNs, &wv);
+        if (lane < S) ok = wait_tagged(dtot + lane, tag, kDepWaitNs, &wv, 64u);
         const bool all_ok = __all_sync(0xFFFFFFFFu, ok);
         if (all_ok) {
           const float rp = lane < S ? __uint_as_float(static_cast<uint32_t>(wv)) : 0.f;
@@ -2074,23 +2093,26 @@ __device__ __forceinline__ void draw_cta(const Args& a, int du, int slice) {
       }
       __syncthreads();
       const bool all_in = sm.all_in != 0;
-      const bool cand = !all_in || sm.tmo != 0 || sm.cstar == slice;
-      if (cand && tid == 0)
+      const bool clean = all_in && sm.tmo == 0;
+      const bool cand = !clean || sm.cstar == slice;
+      // warp 1 claims the row while warp 0 scans the slice for the crossing
+      if (cand && tid == 32)
         sm.own = atomicMax(reinterpret_cast<unsigned int*>(a.draw_owner) + du, tag) < tag ? 1 : 0;
+      if (cand && clean && warp == 0) scan_slice(sm.use_p ? &sm.ps[0][0] : &sm.rs[0][0], true);
       __syncthreads();
       const bool own = cand && sm.own != 0;
       if (!own) {
         leave();
         return;
       }
-      if (all_in && sm.tmo == 0) {
-        if (warp == 0) scan_slice(sm.use_p ? &sm.ps[0][0] : &sm.rs[0][0], true);
-      } else if (tid == 0) {
-        sm.drawn = -1;
-        sm.margin = INFINITY;
-        sm.tmo = 1;
+      if (!clean) {
+        if (tid == 0) {
+          sm.drawn = -1;
+          sm.margin = INFINITY;
+          sm.tmo = 1;
+        }
+        __syncthreads();
       }
-      __syncthreads();
     } else {
       if (tid == 0) sm.is_last = arrive_acq_rel_gpu(a.draw_arrive + du) == S - 1;
       __syncthreads();
