@@ -36,7 +36,7 @@ def short_wait_lib():
     return L
 
 
-@pytest.mark.parametrize("V", [8003, 8000], ids=["two-kernel path", "fused path"])
+@pytest.mark.parametrize("V", [8003, 8000], ids=["unaligned rows", "aligned rows (bulk-copy ring)"])
 def test_short_waits_give_up_and_report(short_wait_lib, V):
     L = short_wait_lib
     w = synth.WORKLOADS["zipf_b16_k5_v32000_bf16"].replace(B=4, V=V)
