@@ -99,18 +99,11 @@ __device__ __forceinline__ void st_release_gpu(int32_t* p, int32_t v) {
 // whole CTA wrote before the barrier (the barrier orders those writes before
 // this thread's), and after the next barrier the acquire makes what the
 // earlier arrivals published visible to the whole CTA.  Returns the old value.
-// Fire-and-forget arrival with release semantics (same publication rule as
-// above); the thread does not wait for the counter's value.
-__device__ __forceinline__ void arrive_release_gpu(int32_t* p) {
-  asm volatile("red.release.gpu.global.add.s32 [%0], 1;" ::"l"(p) : "memory");
-}
-
 __device__ __forceinline__ int32_t arrive_acq_rel_gpu(int32_t* p) {
   int32_t old;
   asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], 1;" : "=r"(old) : "l"(p) : "memory");
   return old;
 }
-
 
 // CTA-scope acquire-release add on a shared-memory counter; returns the old value.
 __device__ __forceinline__ uint32_t atom_add_acq_rel_cta_shared(uint32_t* p, uint32_t v) {
@@ -154,20 +147,6 @@ __device__ __forceinline__ bool wait_tagged(const uint64_t* word, uint32_t tag, 
   return false;
 }
 
-// Bounded wait for a flag written by another CTA (or grid): true once
-// *flag == want; false after `limit_ns` of waiting (or as many polls).
-__device__ __forceinline__ bool wait_flag(const int32_t* flag, int32_t want, unsigned long long limit_ns) {
-  const unsigned long long t0 = global_ns();
-  uint32_t sleep_ns = 64;
-  for (uint32_t i = 0; i < 50000000u; ++i) {
-    if (ld_acquire_gpu(flag) == want) return true;
-    if (global_ns() - t0 > limit_ns) return false;
-    __nanosleep(sleep_ns);
-    if (sleep_ns < 256) sleep_ns <<= 1;
-  }
-  return false;
-}
-
 // 1-D bulk copy global -> this CTA's shared memory (no multicast).  Both
 // addresses 16-byte aligned, bytes a multiple of 16.
 __device__ __forceinline__ void bulk_copy_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
@@ -195,20 +174,6 @@ __device__ __forceinline__ uint64_t l2_policy_evict_first() {
   uint64_t p;
   asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
   return p;
-}
-
-// Split cluster barrier (all threads of every CTA of the cluster): arrive
-// with release semantics, wait with acquire semantics.  Every thread
-// alternates arrive and wait.
-__device__ __forceinline__ void cluster_arrive() {
-  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
-}
-__device__ __forceinline__ void cluster_wait() {
-  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
-__device__ __forceinline__ void cluster_sync_all() {
-  cluster_arrive();
-  cluster_wait();
 }
 
 // ---------------------------------------------------------------------------
@@ -314,12 +279,6 @@ __device__ __forceinline__ int32_t fallback_token(unsigned long long seed, int b
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
-  return v;
-}
-
-__device__ __forceinline__ float warp_max_nan(float v) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v = fmax_nan(v, __shfl_xor_sync(0xFFFFFFFFu, v, o));
   return v;
 }
 

@@ -83,9 +83,6 @@ constexpr float kNearTie = 1e-5f;
 // a row's decision word): 1 s
 constexpr unsigned long long kDepWaitNs = SSD_DEP_WAIT_NS;
 constexpr int kFlagTimeout = SSD_ROW_DEVICE_TIMEOUT;
-#ifndef SSD_LAST_ARRIVES
-#define SSD_LAST_ARRIVES 1  // the last slice / unit to arrive finalises (no waits)
-#endif
 constexpr size_t kRingBytes = static_cast<size_t>(kStages) * 2 * kChunkVecs * 16;
 
 static_assert(8 * (kCandCap + kGatherCap + kSelCap) <= kRingBytes, "merge buffers must fit in the idle ring");
@@ -504,7 +501,6 @@ __device__ __forceinline__ void fanout_row(float alpha_f, int K, int budget, int
   }
 }
 
-
 // Power-law plan ([ZH] section 2 challenge 1, the acceptance's power law;
 // [NL] section 3A, a geometric series): F_k proportional to P(k)^gamma,
 // gamma = q / 8, the optimum when an outcome's hit rate given F guesses
@@ -565,10 +561,6 @@ __device__ __forceinline__ void fanout_row_power(float alpha_f, int K, int budge
     --rem;
   }
 }
-
-#ifndef SSD_RING_WARP_RELEASE
-#define SSD_RING_WARP_RELEASE 1
-#endif
 
 // Ring of bulk copies that streams one slice of up to two rows of a unit
 // through shared memory, chunk by chunk (CV 16-byte vectors per row per
@@ -643,7 +635,6 @@ struct Ring {
     if (tid == 0)
       for (int c = 0; c < min(ST, nch); ++c) issue(c);
   }
-#if SSD_RING_WARP_RELEASE
   // Chunk c is ready for this thread.
   __device__ __forceinline__ void acquire(int c, int tid, int& tmo) {
     if (!mbar_wait_bounded(&full[c % ST], (c / ST) & 1, kRingWaitNs)) tmo = 1;
@@ -666,22 +657,6 @@ struct Ring {
     if (tmo && tid == 0)
       for (int c = max(0, nch - ST); c < nch; ++c) mbar_wait_bounded(&full[c % ST], (c / ST) & 1, kRingWaitNs);
   }
-#else
-  // Chunk c is ready for every thread; the barrier also marks chunk c - 1
-  // consumed, so its stage is refilled.
-  __device__ __forceinline__ void acquire(int c, int tid, int& tmo) {
-    if (tid == 0 && !mbar_wait_bounded(&full[c % ST], (c / ST) & 1, kRingWaitNs)) tmo = 1;
-    __syncthreads();
-    if (tid == 0 && c > 0 && c - 1 + ST < nch) issue(c - 1 + ST);
-    if (tid != 0 && !mbar_try_wait(&full[c % ST], (c / ST) & 1, 0u)) tmo = 1;
-  }
-  __device__ __forceinline__ void release(int, int) {}
-  __device__ __forceinline__ void drain(int tid, int tmo) {
-    if (tmo && tid == 0)
-      for (int c = max(0, n_issued - ST); c < n_issued; ++c)
-        mbar_wait_bounded(&full[c % ST], (c / ST) & 1, kRingWaitNs);
-  }
-#endif
   __device__ __forceinline__ uint4 vec(int c, int r, int tid) const {
     return *reinterpret_cast<const uint4*>(stage(c % ST, r) + tid * 16);
   }
@@ -1214,28 +1189,11 @@ __device__ __forceinline__ void stats_cta(const Args& a, int b, int j, int slice
   }
   __syncthreads();
   if constexpr (kAligned) ring.drain(tid, tmo);
-#if SSD_LAST_ARRIVES
   // The unit's last slice to arrive finalizes; the others leave.  Nobody
   // waits: the arrival is one acquire-release reduction per slice.
   if (tid == 0) sm.is_last = arrive_acq_rel_gpu(a.arrive1 + u) == S - 1 ? 1 : 0;
   __syncthreads();
   if (!sm.is_last) return;
-  const bool arrivals_ok = true;
-#else
-  // The unit's last slice, the last of its CTAs to be scheduled, finalizes:
-  // the others publish and leave without waiting; it waits (bounded) until
-  // they have all published.
-  if (slice != S - 1) {
-    if (tid == 0) arrive_release_gpu(a.arrive1 + u);
-    return;
-  }
-  if (tid == 0) {
-    sm.is_last = wait_flag(a.arrive1 + u, S - 1, kDepWaitNs) ? 1 : 0;
-    if (!sm.is_last) atomicExch(a.error, 1);
-  }
-  __syncthreads();
-  const bool arrivals_ok = sm.is_last != 0;
-#endif
 
   // =============== the unit's finalizer: its last slice, once all have arrived ======
   const SlicePart* parts = a.parts + u * a.n_slices;
@@ -1307,7 +1265,7 @@ __device__ __forceinline__ void stats_cta(const Args& a, int b, int j, int slice
   }
   __syncthreads();
   const float MP = sm.MP, MQ = sm.MQ, SP = sm.SP, SQ = sm.SQ;
-  if (sm.tmo || !arrivals_ok) flags |= kFlagTimeout;
+  if (sm.tmo) flags |= kFlagTimeout;
   // Early exit: when a slice skipped p_j, position j lies past k* and its
   // accept test is not taken (a_j is not reported).
   const bool p_read = verify && sm.pskip == 0;
@@ -1440,26 +1398,10 @@ __device__ __forceinline__ void stats_cta(const Args& a, int b, int j, int slice
     }
     return;
   }
-#if SSD_LAST_ARRIVES
   // Likewise per row: the last unit of the row to arrive decides.
   if (tid == 0) sm.is_last_row = arrive_acq_rel_gpu(a.row_arrive + b) == upr - 1 ? 1 : 0;
   __syncthreads();
   if (!sm.is_last_row) return;
-  const bool row_ok = true;
-#else
-  // Likewise per row: unit j = 0, whose CTAs are the row's last to be
-  // scheduled, decides once the other units have published.
-  if (j != 0) {
-    if (tid == 0) arrive_release_gpu(a.row_arrive + b);
-    return;
-  }
-  if (tid == 0) {
-    sm.is_last_row = wait_flag(a.row_arrive + b, upr - 1, kDepWaitNs) ? 1 : 0;
-    if (!sm.is_last_row) atomicExch(a.error, 1);
-  }
-  __syncthreads();
-  const bool row_ok = sm.is_last_row != 0;
-#endif
 
   // =============== the row's decision: unit j = 0, once all units have arrived ======
   // One warp; lane k reads unit k's record (k = 32 only when K = 32), so the
@@ -1470,7 +1412,6 @@ __device__ __forceinline__ void stats_cta(const Args& a, int b, int j, int slice
     if (lane < upr) fl |= __ldcg(&us[lane].flags);
     if (lane + 32 < upr) fl |= __ldcg(&us[lane + 32].flags);
     fl = static_cast<int>(__reduce_or_sync(0xFFFFFFFFu, static_cast<unsigned>(fl)));
-    if (!row_ok) fl |= kFlagTimeout;
     if (verify) {
       // k* = the first rejected position, else K
       const bool rej = lane < K && __ldcg(&us[lane].rejected) != 0;
