@@ -242,7 +242,7 @@ static WsLayout ws_layout(int B, int K, int V, int dtype) {
   w.rstate = off;      off = up256(off + nb * sizeof(RowState));
   w.rflag = off;       off += nb * static_cast<size_t>(K) * sizeof(uint64_t);  // 8-byte aligned here
   w.uword = off;       off += units * sizeof(uint64_t);
-  w.dtot = off;        off += nb * static_cast<size_t>(K) * ns * sizeof(uint64_t);
+  w.dtot = off;        off += nb * static_cast<size_t>(K) * 2 * ns * sizeof(uint64_t);
   w.arrive1 = off;     off += units * sizeof(int32_t);
   w.row_arrive = off;  off += nb * sizeof(int32_t);
   w.draw_arrive = off; off += nb * static_cast<size_t>(K) * sizeof(int32_t);

@@ -1547,7 +1547,7 @@ struct Smem2 {
   float rs[kMaxChunks][kWarps];
   float ps[kMaxChunks][kWarps];
   int32_t s_F[SSD_MAX_K + 1];
-  float tl, total, margin, myR;
+  float tl, total, margin, myR, myRP;
   int32_t cstar, use_p, drawn, is_last, is_last_row, slot, tmo, all_in, own;
 };
 
@@ -1795,6 +1795,8 @@ __device__ __forceinline__ void draw_cta(const Args& a, int du, int slice) {
   int tmo = 0;
   DrawPart* dparts = a.dparts + static_cast<long long>(du) * S;
   int32_t seg_tok0 = -1, seg_tok1 = -1;  // the last slice: cache segment k*, prefetched
+  bool late_claim = false;   // resident draw: the crossing CTA claims the row after writing it
+  uint32_t claim_tag = 0;
 
   if (streams) {
     // ---- this slice's mass per (chunk, warp), in token order ------------------------
@@ -1834,6 +1836,7 @@ __device__ __forceinline__ void draw_cta(const Args& a, int du, int slice) {
         dparts[slice].RP = RP;
         dparts[slice].timeout = tmo;
         sm.myR = tmo ? __int_as_float(0x7FC00000) : R;
+        sm.myRP = RP;
       }
     }
     if (!resident) {
@@ -1986,10 +1989,13 @@ __device__ __forceinline__ void draw_cta(const Args& a, int du, int slice) {
       // an atomic maximum with the call's tag on the row's owner word lets
       // exactly one CTA write the row.
       const uint32_t tag = *reinterpret_cast<volatile const uint32_t*>(a.epoch) + 1u;
-      uint64_t* const dtot = a.dtot + static_cast<long long>(du) * S;
+      uint64_t* const dtot = a.dtot + static_cast<long long>(du) * 2 * S;
       if (warp == 0) {
+        // the two words carry everything the others read (no release needed):
+        // this slice's residual mass, and its mass of p for a zero residual
         if (lane == 0) {
-          st_release_gpu_u64(dtot + slice, static_cast<uint64_t>(tag) << 32 | __float_as_uint(sm.myR));
+          st_relaxed_gpu_u64(dtot + slice, static_cast<uint64_t>(tag) << 32 | __float_as_uint(sm.myR));
+          st_relaxed_gpu_u64(dtot + S + slice, static_cast<uint64_t>(tag) << 32 | __float_as_uint(sm.myRP));
         }
         uint64_t wv = 0;
         bool ok = true;
@@ -2001,7 +2007,11 @@ __device__ __forceinline__ void draw_cta(const Args& a, int du, int slice) {
           for (int c = 0; c < S; ++c) R += __shfl_sync(0xFFFFFFFFu, rp, c);
           const int use_p = (draw == kDrawResidual && !(R > 0.f) && R == R) ? 1 : 0;
           float pp = 0.f;
-          if (use_p && lane < S) pp = __ldcg(&dparts[lane].RP);  // rare: the row's residual is 0
+          if (use_p) {  // rare: the row's residual is 0
+            uint64_t wp = 0;
+            if (lane < S && wait_tagged(dtot + S + lane, tag, kDepWaitNs, &wp, 64u))
+              pp = __uint_as_float(static_cast<uint32_t>(wp));
+          }
           float RP = 0.f;
           for (int c = 0; c < S; ++c) RP += __shfl_sync(0xFFFFFFFFu, pp, c);
           const float total = use_p ? RP : R;
@@ -2033,20 +2043,26 @@ __device__ __forceinline__ void draw_cta(const Args& a, int du, int slice) {
         }
       }
       __syncthreads();
-      const bool all_in = sm.all_in != 0;
-      const bool clean = all_in && sm.tmo == 0;
-      const bool cand = !clean || sm.cstar == slice;
-      // warp 1 claims the row while warp 0 scans the slice for the crossing
-      if (cand && tid == 32)
-        sm.own = atomicMax(reinterpret_cast<unsigned int*>(a.draw_owner) + du, tag) < tag ? 1 : 0;
-      if (cand && clean && warp == 0) scan_slice(sm.use_p ? &sm.ps[0][0] : &sm.rs[0][0], true);
-      __syncthreads();
-      const bool own = cand && sm.own != 0;
-      if (!own) {
-        leave();
-        return;
-      }
-      if (!clean) {
+      const bool clean = sm.all_in != 0 && sm.tmo == 0;
+      claim_tag = tag;
+      if (clean) {
+        // the slice holding the crossing finishes the row, and claims it
+        // only after writing (a CTA whose wait gave up may have claimed it
+        // first: then the row is rewritten as void)
+        if (sm.cstar != slice) {
+          leave();
+          return;
+        }
+        if (warp == 0) scan_slice(sm.use_p ? &sm.ps[0][0] : &sm.rs[0][0], true);
+        __syncthreads();
+        late_claim = true;
+      } else {
+        if (tid == 0) sm.own = atomicMax(reinterpret_cast<unsigned int*>(a.draw_owner) + du, tag) < tag ? 1 : 0;
+        __syncthreads();
+        if (!sm.own) {
+          leave();
+          return;
+        }
         if (tid == 0) {
           sm.drawn = -1;
           sm.margin = INFINITY;
@@ -2117,7 +2133,8 @@ __device__ __forceinline__ void draw_cta(const Args& a, int du, int slice) {
   }
 
   const int kstar = j;
-  int fl = rowflags | (tmo_all ? kFlagTimeout : 0);
+  auto finish_row = [&](bool void_row) {
+  int fl = rowflags | ((tmo_all || void_row) ? kFlagTimeout : 0);
   const bool invalid = (fl & SSD_ROW_INVALID) != 0;
   if (tid == 0) {
     if (!kGreedy && (amargin < kNearTie || sm.margin < kNearTie)) fl |= SSD_ROW_NEAR_TIE;
@@ -2179,6 +2196,14 @@ __device__ __forceinline__ void draw_cta(const Args& a, int du, int slice) {
         t = fallback_token(a.fallback_seed, b, i, V);
       a.c_next[static_cast<long long>(b) * K + i] = t;
     }
+  }
+  };
+  finish_row(false);
+  if (late_claim) {
+    __syncthreads();
+    if (tid == 0) sm.own = atomicMax(reinterpret_cast<unsigned int*>(a.draw_owner) + du, claim_tag) < claim_tag ? 1 : 0;
+    __syncthreads();
+    if (!sm.own) finish_row(true);  // a CTA whose wait gave up claimed the row first
   }
   leave();
 }
