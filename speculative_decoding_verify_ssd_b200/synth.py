@@ -123,7 +123,7 @@ class Workload:
     budget: int
     C: float
     seed: int
-    alpha: float            # fan-out acceptance estimate (mean overlap, see DESIGN)
+    alpha: float            # fan-out acceptance estimate: the mean overlap sum(min(p, q)), calibrated offline
     fallback_seed: int
     fanout_mode: int = 0    # 0 geometric, 1 uniform
 
