@@ -84,16 +84,6 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
   return false;
 }
 
-// Acquire load / release store of a flag in global memory, GPU scope.
-__device__ __forceinline__ int32_t ld_acquire_gpu(const int32_t* p) {
-  int32_t v;
-  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-  return v;
-}
-__device__ __forceinline__ void st_release_gpu(int32_t* p, int32_t v) {
-  asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
-}
-
 // One thread's arrival on a counter in global memory, GPU scope, acquire and
 // release at once.  Issued after a CTA barrier, the release publishes what the
 // whole CTA wrote before the barrier (the barrier orders those writes before
