@@ -410,6 +410,7 @@ static ssd_status verify_impl(const void* target_logits, const void* draft_logit
   if (dtype != SSD_DTYPE_BF16 && dtype != SSD_DTYPE_FP32) return SSD_ERR_DTYPE;
   if (B < 0 || K < 1 || K > SSD_MAX_K || V < 1) return SSD_ERR_INVALID_ARG;
   if (!(T >= 0.f) || isinf(T)) return SSD_ERR_INVALID_ARG;
+  if (B == 0) return SSD_OK;  // nothing to do (empty tensors may carry null pointers)
   const bool has_plan = F != nullptr || alpha != nullptr;
   if (has_plan && (!(C > 0.f && C <= 1.f) || budget < 0 || budget > SSD_MAX_BUDGET || budget > V))
     return SSD_ERR_INVALID_ARG;
@@ -417,7 +418,6 @@ static ssd_status verify_impl(const void* target_logits, const void* draft_logit
     return SSD_ERR_INVALID_ARG;
   if (cache && (!has_plan || !cache->offsets || !cache->tokens || !cache->hit || !cache->slot || !cache->next_tokens))
     return SSD_ERR_INVALID_ARG;
-  if (B == 0) return SSD_OK;
   if (!target_logits || !draft_logits || !draft_tokens || !uniforms || !n_accepted || !bonus || !out_tokens ||
       !accept_prob || !residual_mass || !status)
     return SSD_ERR_INVALID_ARG;

@@ -22,6 +22,7 @@ SMALL = [
     ("tiny_b1_k4_v1024_fp32", {}),
     ("zipf_b16_k5_v32000_bf16", {"T": 0.0, "seed": 22}),    # greedy
     ("zipf_b64_k6_v128256_bf16", {"B": 24, "seed": 23}),
+    ("zipf_b16_k5_v32000_bf16", {"B": 6, "K": 32, "V": 4096, "budget": 512, "seed": 32}),  # largest K and budget
 ]
 
 

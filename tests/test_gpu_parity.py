@@ -12,7 +12,7 @@ import oracle
 from speculative_decoding_verify_ssd_b200 import binding as ssd
 from speculative_decoding_verify_ssd_b200 import synth
 
-from ssd_testlib import Case, check_row_properties, compare, to_dev, PROB_ATOL, LSE_RTOL
+from ssd_testlib import Case, check_row_properties, compare, draft_tokens_for, to_dev, PROB_ATOL, LSE_RTOL
 
 pytestmark = pytest.mark.gpu
 
@@ -195,6 +195,38 @@ def test_F_zero_budget_K_plus_1_and_C_one():
     gpu = case.run_gpu()
     orc = case.run_oracle()
     compare(case, gpu, orc)
+
+
+def test_max_draft_length_and_max_budget():
+    """K = 32, the largest draft length (its unit 32 rides in the second word
+    a lane of the draw's decision wait holds), with the largest budget, 512
+    (top-F sets above a slice's candidate slots take the exact global
+    path).  Rows 0 and 1 have draft rows equal to their target rows and
+    C = 1, so every position is accepted and the bonus comes from p_K."""
+    w = W["zipf_b16_k5_v32000_bf16"].replace(B=4, K=32, V=4096, budget=512, C=1.0, seed=31)
+    case = Case(w)
+    for b in (0, 1):
+        case.g["draft"][b] = case.g["target"][b, :w.K]
+    case.tokens = draft_tokens_for(w, case.g, case.F)
+    gpu = case.run_gpu()
+    orc = case.run_oracle()
+    assert list(orc["n_accepted"][:2]) == [32, 32]
+    compare(case, gpu, orc)
+    check_row_properties(case, gpu)
+
+
+def test_empty_batch():
+    """B = 0: the call succeeds, launches nothing and returns empty outputs."""
+    w = W["zipf_b16_k5_v32000_bf16"]
+    dev = torch.device("cuda")
+    t = torch.zeros(0, w.K + 1, w.V, dtype=torch.bfloat16, device=dev)
+    d = torch.zeros(0, w.K, w.V, dtype=torch.bfloat16, device=dev)
+    tok = torch.zeros(0, w.K, dtype=torch.int32, device=dev)
+    u = torch.zeros(0, w.K + 1, dtype=torch.float32, device=dev)
+    F = torch.zeros(0, w.K + 1, dtype=torch.int32, device=dev)
+    r = ssd.ssd_verify(t, d, tok, u, w.T, F=F, C_coef=w.C, budget=w.budget, cache=True)
+    torch.cuda.synchronize()
+    assert r.n_accepted.numel() == 0 and r.bonus.numel() == 0 and r.status.numel() == 0
 
 
 def test_single_row_and_max_vocab():
