@@ -13,6 +13,7 @@
 #include "../../include/ssd.h"
 #include "ssd_device.cuh"
 #include "ssd_kernels.cuh"
+#include "ssd_cluster.cuh"
 
 namespace ssd {
 
@@ -275,7 +276,9 @@ static void bind_workspace(Args& a, void* ws, const WsLayout& w) {
   a.k2_done = reinterpret_cast<int32_t*>(base + w.k2_done);
   a.error = reinterpret_cast<int32_t*>(base + w.error);
   a.skipped = reinterpret_cast<unsigned long long*>(base + w.skipped);
+  a.uout = reinterpret_cast<UnitOut*>(base + w.ustate);  // the cluster form's unit records
 }
+static_assert(sizeof(UnitOut) <= sizeof(UnitState), "a unit record of the cluster form fits a unit state");
 
 template <typename TIn, bool kAligned, bool kGreedy>
 static ssd_status launch_t(const Args& a, long long units, long long draw_units, cudaStream_t stream) {
@@ -323,6 +326,82 @@ static ssd_status launch(const Args& a, int dtype, bool aligned, long long units
                   : launch_t<float, true, false>(a, units, draw_units, stream);
   return greedy ? launch_t<float, false, true>(a, units, draw_units, stream)
                 : launch_t<float, false, false>(a, units, draw_units, stream);
+}
+
+// ---------------------------------------------------------------------------
+// The cluster form (ssd_cluster.cuh): bf16 rows of a multiple of 8 tokens,
+// T > 0, budgets up to kClCandCap.  Built in with SSD_CLUSTER_VERIFY=1; the
+// default build runs every verify call in the two-kernel form, which measures
+// faster on B200 (the cluster form's draws hold their CTAs' slots through a
+// second pass over the slice, so fewer CTAs stream at a time).
+// ---------------------------------------------------------------------------
+#ifndef SSD_CLUSTER_VERIFY
+#define SSD_CLUSTER_VERIFY 0
+#endif
+
+#ifndef SSD_CL_CARVEOUT
+#define SSD_CL_CARVEOUT 100  // percent of the SM's unified L1 / shared storage asked for as shared memory
+#endif
+
+static std::map<std::tuple<int, int, size_t>, int> g_cl_ready;
+
+// Clusters of CS CTAs with `smem` dynamic bytes each that the current device
+// can hold at once (0: the form is not available, and ssd_verify uses the
+// two-kernel form instead).  Looked up once per (device, CS, smem).
+static int cluster_ready(int CS, size_t smem) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  std::lock_guard<std::mutex> lock(g_attr_mu);
+  const auto key = std::make_tuple(dev, CS, smem);
+  const auto it = g_cl_ready.find(key);
+  if (it != g_cl_ready.end()) return it->second;
+  const void* fn = reinterpret_cast<const void*>(&ssd_cluster_kernel);
+  int n = 0;
+  bool ok = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kRingBytes)) ==
+            cudaSuccess;
+  if (ok && CS > 8) ok = cudaFuncSetAttribute(fn, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess;
+  // five CTAs of ~43 KB per SM need the largest shared-memory carveout
+  if (ok && SSD_CL_CARVEOUT >= 0)
+    ok = cudaFuncSetAttribute(fn, cudaFuncAttributePreferredSharedMemoryCarveout, SSD_CL_CARVEOUT) == cudaSuccess;
+  if (ok) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(CS));
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeClusterDimension;
+    at[0].val.clusterDim.x = static_cast<unsigned>(CS);
+    at[0].val.clusterDim.y = 1;
+    at[0].val.clusterDim.z = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    if (cudaOccupancyMaxActiveClusters(&n, fn, &cfg) != cudaSuccess) n = 0;
+  }
+  if (!ok || n <= 0) {
+    (void)cudaGetLastError();  // a refused attribute leaves no sticky error behind
+    n = 0;
+  }
+  g_cl_ready[key] = n;
+  return n;
+}
+
+static ssd_status launch_cluster(const Args& a, long long units, cudaStream_t stream) {
+  const long long grid = units * a.cl_size;
+  if (grid > 0x7FFFFFFFLL) return SSD_ERR_INVALID_ARG;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid));
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = kRingBytes;  // the bulk-copy ring
+  cfg.stream = stream;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeClusterDimension;
+  at[0].val.clusterDim.x = static_cast<unsigned>(a.cl_size);
+  at[0].val.clusterDim.y = 1;
+  at[0].val.clusterDim.z = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, ssd_cluster_kernel, a) != cudaSuccess) return SSD_ERR_CUDA;
+  return SSD_OK;
 }
 
 static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -469,7 +548,17 @@ static ssd_status verify_impl(const void* target_logits, const void* draft_logit
   }
   bind_workspace(a, workspace, wl);
   const int VE = 16 / esize;
-  return launch(a, dtype, V % VE == 0, units, B, static_cast<cudaStream_t>(stream));
+  const bool aligned = V % VE == 0;
+  if (SSD_CLUSTER_VERIFY && !early_exit && dtype == SSD_DTYPE_BF16 && aligned && T > 0.f &&
+      (!has_plan || budget <= kClCandCap)) {
+    // one cluster per unit, one CTA per slice of the statistics plan
+    if (cluster_ready(plan.n_slices, kRingBytes) > 0) {
+      a.cl_size = plan.n_slices;
+      a.cl_len = plan.chunk;
+      return launch_cluster(a, units, static_cast<cudaStream_t>(stream));
+    }
+  }
+  return launch(a, dtype, aligned, units, B, static_cast<cudaStream_t>(stream));
 }
 }  // namespace ssd
 

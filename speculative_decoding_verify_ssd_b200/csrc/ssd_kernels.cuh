@@ -134,6 +134,8 @@ struct RowState {
   int32_t bi, argP;
 };
 
+struct UnitOut;  // ssd_cluster.cuh
+
 struct Args {
   const void* target;      // [B, K+1, V]
   const void* draft;       // [B, K, V]
@@ -188,6 +190,10 @@ struct Args {
   int32_t* k2_done;        // kernel 2 CTAs past their wait
   int32_t* error;
   unsigned long long* skipped;  // early exit: target-row bytes not read
+  // the one-pass cluster form (ssd_cluster.cuh)
+  int cl_size;             // CTAs per unit (the cluster's size)
+  int cl_len;              // tokens of a row per CTA (a multiple of 8)
+  UnitOut* uout;           // per unit: the record its leader publishes
 };
 
 template <typename TIn>

@@ -1,6 +1,9 @@
 """Failure detection on the GPU without a fault: a test build of the library
 whose waits for another CTA's result (a slice partial, a unit record, a row's
-decision word) give up after 200 ns instead of 1 s.  The waits then run out
+decision word) give up after 200 ns instead of 1 s.  Only the two-kernel
+form (the default) has such waits; the optional cluster form's CTAs meet at
+hardware cluster barriers and never poll another CTA's flag, so the test
+build names the two-kernel form explicitly.  The waits then run out
 on an ordinary call; the call must still return, the rows whose waits gave up
 must carry SSD_ROW_DEVICE_TIMEOUT with the void-row outputs, and the
 workspace's error word must read SSD_ERR_TIMEOUT.  The waits on the CTA's own
@@ -25,7 +28,7 @@ SSD_ERR_TIMEOUT = 6
 
 @pytest.fixture(scope="module")
 def short_wait_lib():
-    path = _build.build_variant("shortwait", ["SSD_DEP_WAIT_NS=200ull"])
+    path = _build.build_variant("shortwait", ["SSD_DEP_WAIT_NS=200ull", "SSD_CLUSTER_VERIFY=0"])
     L = C.CDLL(path)
     vp, i32, f32, sz = C.c_void_p, C.c_int, C.c_float, C.c_size_t
     L.ssd_verify.restype = i32
