@@ -1673,32 +1673,57 @@ __device__ __forceinline__ void draw_cta(const Args& a, int du, int slice) {
 
   // ---- the row decision this CTA needs (kernel 1 may still be running) -------------
   if (verify) {
-    // Lane k waits for unit k's tagged word (lane 0 also for unit 32 when
-    // K = 32); k* is the first rejected position, else K.
+    // Lane k polls unit k's tagged word (lane 0 also unit 32's when K = 32).
+    // k* is fixed as soon as the words of positions 0..j are in with j the
+    // first rejected one (or all K+1 words are in, none rejected): the stream
+    // of unit k* starts then, and the words past k* are awaited only before
+    // the row's flags are written (finish_row).
     if (warp == 0) {
-      const uint32_t epoch = *reinterpret_cast<volatile const uint32_t*>(a.epoch);
+      const uint32_t tag = *reinterpret_cast<volatile const uint32_t*>(a.epoch) + 1u;
       const int upr = K + 1;
       const uint64_t* uw = a.uword + static_cast<long long>(du) * upr;
       uint64_t w0 = 0, w1 = 0;
-      bool ok = true;
-      if (lane < upr) ok = wait_tagged(uw + lane, epoch + 1u, kDepWaitNs, &w0, 128u);
-      if (lane + 32 < upr) ok = wait_tagged(uw + lane + 32, epoch + 1u, kDepWaitNs, &w1) && ok;
-      const bool all_ok = __all_sync(0xFFFFFFFFu, ok);
-      const uint32_t lo0 = static_cast<uint32_t>(w0), lo1 = static_cast<uint32_t>(w1);
-      const unsigned rm = __ballot_sync(0xFFFFFFFFu, lane < K && ((lo0 >> 16) & 1u));
-      const int kstar = rm ? __ffs(rm) - 1 : K;
-      // flags of every unit; a near-tie accept test only up to k*; with the
-      // early-exit schedule a non-finite target row and q'(d) = 0 only up to
-      // k* and at K (unit 32 is K itself)
-      uint32_t f = (lo0 | lo1) & 0xFFu;
-      if (!a.early_exit || lane <= kstar || lane == K) f |= (lo0 >> 8) & 0xFFu;
-      f |= (lo1 >> 8) & 0xFFu;
-      if (lane <= kstar && ((lo0 >> 17) & 1u)) f |= SSD_ROW_NEAR_TIE;
+      bool have0 = lane >= upr, have1 = lane + 32 >= upr;
+      int kstar = -1;
+      const unsigned long long t0 = global_ns();
+      uint32_t sleep_ns = 32;
+      for (uint32_t it = 0; it < 50000000u; ++it) {
+        if (!have0) {
+          const uint64_t v = ld_acquire_gpu_u64(uw + lane);
+          if (static_cast<uint32_t>(v >> 32) == tag) { w0 = v; have0 = true; }
+        }
+        if (!have1) {
+          const uint64_t v = ld_acquire_gpu_u64(uw + lane + 32);
+          if (static_cast<uint32_t>(v >> 32) == tag) { w1 = v; have1 = true; }
+        }
+        const unsigned pres = __ballot_sync(0xFFFFFFFFu, have0);
+        const unsigned rm = __ballot_sync(0xFFFFFFFFu, have0 && lane < K && ((static_cast<uint32_t>(w0) >> 16) & 1u));
+        const bool all1 = __all_sync(0xFFFFFFFFu, have1);
+        if (rm) {
+          const int js = __ffs(rm) - 1;
+          const unsigned below = (1u << js) - 1u;
+          if ((pres & below) == below) { kstar = js; break; }
+        } else if (pres == 0xFFFFFFFFu && all1) {
+          kstar = K;
+          break;
+        }
+        if (global_ns() - t0 > kDepWaitNs) break;
+        __nanosleep(sleep_ns);
+        if (sleep_ns < 128u) sleep_ns <<= 1;
+      }
+      const bool ok = kstar >= 0;
+      // flags of the units 0..k* only (every CTA of the row has read the
+      // same words up to k*, so all take the same stream decision); the
+      // flags past k* are added in finish_row
+      const uint32_t lo0 = (have0 && lane <= kstar) ? static_cast<uint32_t>(w0) : 0u;
+      const uint32_t lo1 = (have1 && lane + 32 <= kstar) ? static_cast<uint32_t>(w1) : 0u;
+      uint32_t f = ((lo0 | lo1) & 0xFFu) | ((lo0 >> 8) & 0xFFu) | ((lo1 >> 8) & 0xFFu);
+      if ((lo0 >> 17) & 1u) f |= SSD_ROW_NEAR_TIE;
       f = __reduce_or_sync(0xFFFFFFFFu, f);
       if (lane == 0) {
-        sm.dep_ok = all_ok ? 1 : 0;
-        if (!all_ok) atomicExch(a.error, 1);
-        sm.w_kstar = kstar;
+        sm.dep_ok = ok ? 1 : 0;
+        if (!ok) atomicExch(a.error, 1);
+        sm.w_kstar = ok ? kstar : K;
         sm.w_flags = static_cast<int32_t>(f);
       }
     }
@@ -2139,7 +2164,35 @@ __device__ __forceinline__ void draw_cta(const Args& a, int du, int slice) {
   }
 
   const int kstar = j;
+  bool flags_final = !dep_ok;  // a row whose decision never came is void anyway
   auto finish_row = [&](bool void_row) {
+  if (!flags_final) {
+    // every unit's word (bounded): the flags of the units past k*
+    if (warp == 0) {
+      const uint32_t tag = *reinterpret_cast<volatile const uint32_t*>(a.epoch) + 1u;
+      const int upr = K + 1;
+      const uint64_t* uw = a.uword + static_cast<long long>(b) * upr;
+      uint64_t w0 = 0, w1 = 0;
+      bool ok = true;
+      if (lane < upr) ok = wait_tagged(uw + lane, tag, kDepWaitNs, &w0, 128u);
+      if (lane + 32 < upr) ok = wait_tagged(uw + lane + 32, tag, kDepWaitNs, &w1) && ok;
+      const bool all_ok = __all_sync(0xFFFFFFFFu, ok);
+      const uint32_t lo0 = static_cast<uint32_t>(w0), lo1 = static_cast<uint32_t>(w1);
+      uint32_t f = (lo0 | lo1) & 0xFFu;
+      if (!a.early_exit || lane <= kstar || lane == K) f |= (lo0 >> 8) & 0xFFu;
+      f |= (lo1 >> 8) & 0xFFu;
+      if (lane <= kstar && ((lo0 >> 17) & 1u)) f |= SSD_ROW_NEAR_TIE;
+      f = __reduce_or_sync(0xFFFFFFFFu, f);
+      if (!all_ok) f |= kFlagTimeout;
+      if (lane == 0) {
+        if (!all_ok) atomicExch(a.error, 1);
+        sm.w_flags = static_cast<int32_t>(f);
+      }
+    }
+    __syncthreads();
+    rowflags = sm.w_flags;
+    flags_final = true;
+  }
   int fl = rowflags | ((tmo_all || void_row) ? kFlagTimeout : 0);
   const bool invalid = (fl & SSD_ROW_INVALID) != 0;
   if (tid == 0) {
