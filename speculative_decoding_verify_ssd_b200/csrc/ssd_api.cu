@@ -525,6 +525,12 @@ static ssd_status verify_impl(const void* target_logits, const void* draft_logit
   a.n_slices = plan.n_slices; a.chunk = plan.chunk;
   if (stats_grid(a) > 0x7FFFFFFFLL) return SSD_ERR_INVALID_ARG;
   a.early_exit = early_exit;
+  // Unit K of every row after all positions j < K, when those CTAs fit one
+  // wave of resident statistics CTAs: then the rows are drawn while the short
+  // unit-K CTAs stream.  With more, the rows' finishing draw CTAs would wait
+  // through several waves for unit K's flags, holding their slots.
+  a.k_last = (!early_exit && static_cast<long long>(B) * plan.n_slices <= static_cast<long long>(kMinBlocks) * sm_count())
+                 ? 1 : 0;
   if (early_exit) {
     // the lag: about the rows whose CTAs are scheduled while one position's
     // CTAs stream and finalise (SSD_EE_LAG_PCT % of a wave of resident CTAs)

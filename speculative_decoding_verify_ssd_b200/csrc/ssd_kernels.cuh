@@ -24,7 +24,8 @@
 //   accept test a_j = min(1, p_j(d_j) / q'_j(d_j)); in the same way unit
 //   j = 0, the row's last to be scheduled, fixes k*, the first rejected
 //   position, and publishes the row's decision word (call epoch, k*, flags).
-//   Rows are taken in order, so they are decided one after another.
+//   Units are taken row by row, positions j < K of every row before any
+//   row's unit K, so rows are decided one after another.
 //
 // Kernel 2 (draw): one CTA per (row, slice) of the single unit each row
 //   draws from: the residual r = max(0, p_k* - q'_k*) (or p_K after full
@@ -152,6 +153,7 @@ struct Args {
   int draws;               // kernel 2 runs (verify always; reweight: draft tokens drawn)
   int early_exit;          // verify: the early-exit read schedule
   int lag;                 // early exit: rows between the CTAs of position j and j + 1
+  int k_last;              // verify, full read: every row's unit K after all positions j < K
   float T, C;
   // verify outputs
   int32_t* n_accepted;
@@ -1538,6 +1540,19 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) ssd_stats_kernel(const _
     __syncthreads();
     b = s_unit[0];
     j = s_unit[1];
+  } else if (a.k_last) {
+    // positions j < K of every row first (row by row), then every row's
+    // unit K: a row's k* is fixed by its positions up to the first rejection,
+    // so most rows are drawn while the short unit-K CTAs (one row each) still
+    // stream (the host asks for it when those CTAs fit one wave)
+    const int nfirst = a.B * a.K;
+    if (order < nfirst) {
+      b = order / a.K;
+      j = order % a.K;
+    } else {
+      b = order - nfirst;
+      j = a.K;
+    }
   }
   // kernel 2 may be scheduled once every CTA of this grid has started; it
   // waits for each of its units' records on its own
@@ -1549,7 +1564,7 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) ssd_stats_kernel(const _
 struct Smem2 {
   uint64_t full[kStages];
   uint32_t rel[kStages];
-  int32_t dep_ok, w_kstar, w_flags;
+  int32_t dep_ok, w_kstar, w_flags, w_final, w_flags_all;
   float rs[kMaxChunks][kWarps];
   float ps[kMaxChunks][kWarps];
   int32_t s_F[SSD_MAX_K + 1];
@@ -1720,11 +1735,22 @@ __device__ __forceinline__ void draw_cta(const Args& a, int du, int slice) {
       uint32_t f = ((lo0 | lo1) & 0xFFu) | ((lo0 >> 8) & 0xFFu) | ((lo1 >> 8) & 0xFFu);
       if ((lo0 >> 17) & 1u) f |= SSD_ROW_NEAR_TIE;
       f = __reduce_or_sync(0xFFFFFFFFu, f);
+      // when every word was already in, the row's final flags too (as
+      // finish_row would form them), so the finishing CTA need not read again
+      const bool all_in = __all_sync(0xFFFFFFFFu, have0 && have1);
+      const uint32_t a0 = static_cast<uint32_t>(w0), a1 = static_cast<uint32_t>(w1);
+      uint32_t ff = (a0 | a1) & 0xFFu;
+      if (!a.early_exit || lane <= kstar || lane == K) ff |= (a0 >> 8) & 0xFFu;
+      ff |= (a1 >> 8) & 0xFFu;
+      if (lane <= kstar && ((a0 >> 17) & 1u)) ff |= SSD_ROW_NEAR_TIE;
+      ff = __reduce_or_sync(0xFFFFFFFFu, ff);
       if (lane == 0) {
         sm.dep_ok = ok ? 1 : 0;
         if (!ok) atomicExch(a.error, 1);
         sm.w_kstar = ok ? kstar : K;
         sm.w_flags = static_cast<int32_t>(f);
+        sm.w_final = (ok && all_in) ? 1 : 0;
+        sm.w_flags_all = static_cast<int32_t>(ff);
       }
     }
   } else if (tid == 0) {
@@ -2165,6 +2191,10 @@ __device__ __forceinline__ void draw_cta(const Args& a, int du, int slice) {
 
   const int kstar = j;
   bool flags_final = !dep_ok;  // a row whose decision never came is void anyway
+  if (verify && dep_ok && sm.w_final) {  // every word was in when k* was taken
+    rowflags = sm.w_flags_all;
+    flags_final = true;
+  }
   auto finish_row = [&](bool void_row) {
   if (!flags_final) {
     // every unit's word (bounded): the flags of the units past k*
