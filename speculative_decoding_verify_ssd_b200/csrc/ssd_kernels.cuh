@@ -11,33 +11,35 @@
 //   [NL] = the Dutch edition, sections 2 and 3A-3C):
 //     - online max and rescaled sum of exp2 of p_j and q_j (temperature
 //       softmax, one exp per element), or the greedy argmax when T = 0;
-//     - the top two vector maxima of the top-F source row (q_j) and the vector
-//       holding the larger, so the slice's own top-F (which contains the
+//     - the three largest vector maxima of the top-F source row (q_j) and the
+//       two vectors holding the largest, so the slice's own top-F (which contains the
 //       slice's share of the unit's top-F, [ZH] challenge 2 "top-F tokens")
 //       comes from registers: the F-th largest thread maximum bounds it from
 //       below.
 //   It publishes a small partial and leaves (one thread's release reduction
-//   on the unit's counter).  The unit's last slice, its last CTA to be
-//   scheduled, waits for the others, merges the partials, selects the exact
+//   on the unit's counter).  The unit's last slice to arrive (nobody waits)
+//   merges the partials, selects the exact
 //   top-F by (logit desc, token id asc), forms Q_S and the Saguaro normaliser
 //   Z = 1 - (1 - C) Q_S ([ZH] challenge 2; [NL] 3B), and runs the lossless
-//   accept test a_j = min(1, p_j(d_j) / q'_j(d_j)); in the same way unit
-//   j = 0, the row's last to be scheduled, fixes k*, the first rejected
-//   position, and publishes the row's decision word (call epoch, k*, flags).
-//   Units are taken row by row, positions j < K of every row before any
-//   row's unit K, so rows are decided one after another.
+//   accept test a_j = min(1, p_j(d_j) / q'_j(d_j)).  In verify mode it
+//   publishes the unit's result in one tagged word (call epoch, rejected,
+//   near-tie, flags) and nobody waits for the rest of the row; in reweight
+//   mode the row's last unit to finish publishes the row's per-position words.
+//   Units are taken row by row; in verify mode, when every row's unit-K CTAs
+//   fit one wave, positions j < K of every row come before any row's unit K.
 //
 // Kernel 2 (draw): one CTA per (row, slice) of the single unit each row
 //   draws from: the residual r = max(0, p_k* - q'_k*) (or p_K after full
 //   acceptance, or q' for a draft draw).  It is a programmatic dependent of
-//   kernel 1 (scheduled once every kernel-1 CTA has started) and each CTA
-//   waits only for its own row's decision word, so the draws of early rows
-//   run while kernel 1 finishes.  Each CTA sums its slice of r per
-//   (ring chunk, warp); the last CTA of the row finds where the cumulative
-//   mass crosses u * R in token order (slice, chunk, warp, then one re-read
-//   vector per lane), draws the bonus token, and finishes the row: outputs,
-//   the cache lookup of (k*, bonus) and the random-token fallback ([ZH]
-//   basic flow steps 3-4 and challenge 3; [NL] 3C).
+//   kernel 1 (scheduled once every kernel-1 CTA has started).  Each CTA polls
+//   its own row's unit words and takes k* as soon as positions 0..k* are in
+//   (the first rejected one, every earlier one accepted), so the draws of
+//   early rows run while kernel 1 finishes.  Each CTA sums its slice of r per
+//   (ring chunk, warp); the CTA holding the crossing of u * R in token order
+//   (slice, chunk, warp, lane, token) draws the bonus token, reads the words
+//   past k* for the row's flags when it has not seen them yet, and finishes
+//   the row: outputs, the cache lookup of (k*, bonus) and the random-token
+//   fallback ([ZH] basic flow steps 3-4 and challenge 3; [NL] 3C).
 #pragma once
 
 #include <limits.h>
