@@ -203,6 +203,10 @@ ssd_status ssd_saguaro_reweight(const void* draft_logits, int dtype, int B, int 
  *   (R at k* < K, sum of p_K after full acceptance, 1 when T = 0), status [B].
  *   cache: NULL, or a host pointer to an ssd_cache of device pointers.
  *   workspace: as for ssd_saguaro_reweight.
+ *   A build of the library with SSD_CLUSTER_VERIFY=1 runs the calls with
+ *   bf16 logits, rows of a multiple of 8 tokens, T > 0 and budget <= 256 as
+ *   one kernel of thread-block clusters (one cluster per row and position);
+ *   arguments, outputs and error behaviour are the same.
  */
 ssd_status ssd_verify(const void* target_logits, const void* draft_logits, const void* draft_next,
                       int dtype, int B, int K, int V, const int32_t* draft_tokens,
